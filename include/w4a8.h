@@ -1,0 +1,178 @@
+/*
+ * w4a8.h -- C ABI of the asym_w4a8_int8 ConvRot linear layer on NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer computes y = x * W_hat^T where
+ *   - x[M, K] are bf16 activations, rotated per 256-block of K by the
+ *     normalised Sylvester Hadamard matrix H_256 / 16 and quantised to int8
+ *     per token (symmetric absmax / 127, round half to even);
+ *   - W_hat[n, k] = codebook[idx[n, k]] * s_rel[n, k / 16] * s_channel[n] is
+ *     the weight in the same rotated basis, rebuilt from four stored tensors:
+ *     packed 4-bit indices, fp8 e4m3 group scales (one per 16 values), fp32
+ *     row scales and a 16-entry fp32 codebook.
+ * Sources: "Qwen3.8-27B-AEON-ULTIMATE-UNCENSORED-BF16 -- W4A8 ConvRot for
+ * ComfyUI" model card, sections "Why this exists" and "Format" (the four
+ * tensors, three tiers of scaling, rotation group 256, codebook group 16);
+ * "Qwen3.8-27B-W4A8" model card, section "Model Overview" (group sizes,
+ * int8 activations, per-group fp8 scales, fp32 channel scales).
+ *
+ * Conventions for every call below:
+ *   - All buffer pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates no device memory and keeps no reference to any
+ *     buffer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Work is enqueued on it asynchronously; no call synchronises
+ *     except w4a8_get_device_error.
+ *   - Arguments are checked on the host before anything is launched.  On a
+ *     failed check nothing is launched and the status says why.
+ *   - Shapes: K must be a multiple of 256 (the rotation block; a layer whose
+ *     input width is not, such as 4304 = 16 x 269, stays unquantised on the
+ *     pages) and at most W4A8_MAX_K; N must be a positive multiple of 16;
+ *     M must be positive.
+ *   - Every pointer must be 16-byte aligned.
+ *   - The calls run on the current CUDA device, which must be sm_100.
+ */
+#ifndef W4A8_H_
+#define W4A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4A8_ROT_BLOCK 256   /* rotation block along K */
+#define W4A8_GROUP 16        /* values per fp8 group scale */
+#define W4A8_LEVELS 16       /* codebook entries */
+#define W4A8_MAX_K 32768     /* largest supported K */
+
+typedef enum w4a8_status {
+  W4A8_OK = 0,
+  W4A8_ERR_NULL = 1,       /* a required pointer is NULL */
+  W4A8_ERR_SHAPE = 2,      /* M, N or K outside the rules above */
+  W4A8_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned */
+  W4A8_ERR_WORKSPACE = 4,  /* a buffer is smaller than the size function says */
+  W4A8_ERR_CUDA = 5,       /* a CUDA call failed (launch or device query) */
+  W4A8_ERR_TIMEOUT = 6,    /* a bounded device wait gave up (see get_device_error) */
+  W4A8_ERR_ARCH = 7        /* the current device is not sm_100 */
+} w4a8_status;
+
+/*
+ * Size in bytes of the device layout produced by w4a8_pack_layout for an
+ * [N, K] weight, or 0 if (N, K) break the shape rules.  About 0.5625 bytes
+ * per weight (0.5 for the indices, 1/16 for the group scales) plus 4 bytes
+ * per row and 64 bytes for the codebook, each region padded to 256 bytes.
+ */
+size_t w4a8_packed_bytes(int64_t N, int64_t K);
+
+/*
+ * Re-lay the four stored tensors of one layer into the library's device
+ * layout (ConvRot card, "Format": the four tensors of a quantised layer).
+ *   idx        [N, K/2] uint8, row-major.  Byte c of row n holds the index
+ *              of k = 2c in its low nibble and of k = 2c + 1 in its high
+ *              nibble ("packed int4 indices, two per byte").
+ *   s_rel      [N, K/16] uint8, row-major: e4m3fn bit patterns, one per
+ *              group of 16 consecutive k.
+ *   s_channel  [N] fp32: one scale per output row.
+ *   codebook   [16] fp32: the levels the indices point into.
+ *   packed     output, `packed_bytes` >= w4a8_packed_bytes(N, K).  Its
+ *              content is opaque; it is read by w4a8_unpack_dequant and
+ *              w4a8_linear.
+ * Errors: NULL, SHAPE, ALIGN, WORKSPACE (packed_bytes too small), CUDA.
+ */
+w4a8_status w4a8_pack_layout(const uint8_t* idx, const uint8_t* s_rel,
+                             const float* s_channel, const float* codebook,
+                             int64_t N, int64_t K, void* packed,
+                             size_t packed_bytes, void* stream);
+
+/*
+ * Rebuild the weight in the rotated basis (ConvRot card, "Format": "three
+ * tiers of scaling -- codebook shape, group magnitude, row magnitude"):
+ *   w_hat[n, k] = fp32(fp32(codebook[idx[n,k]] * s_rel[n, k/16]) * s_channel[n])
+ * with both products rounded to nearest even (bit-exact).
+ *   packed  a buffer filled by w4a8_pack_layout for the same (N, K).
+ *   w_hat   output [N, K] fp32, row-major.
+ * Errors: NULL, SHAPE, ALIGN, CUDA.
+ */
+w4a8_status w4a8_unpack_dequant(const void* packed, int64_t N, int64_t K,
+                                float* w_hat, void* stream);
+
+/*
+ * Rotate and quantise activations (ConvRot card, "Format": group-wise
+ * Hadamard rotation, group 256; "Qwen3.8-27B-W4A8" card, "Model Overview":
+ * int8 activations):
+ *   x_rot[m, 256b + j] = (1/16) * sum_i x[m, 256b + i] * H_256[i, j]
+ *   s_x[m]             = max_k |x_rot[m, k]| / 127           (fp32)
+ *   x_q[m, k]          = clamp(round_half_even(x_rot / s_x), -127, 127)
+ * The rotation runs in fp32; an all-zero token gives s_x = 0 and x_q = 0.
+ *   x    [M, K] bf16 bit patterns (uint16), row-major.
+ *   x_q  output [M, K] int8, row-major.
+ *   s_x  output [M] fp32.
+ * Errors: NULL, SHAPE, ALIGN, CUDA.
+ */
+w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K,
+                                  int8_t* x_q, float* s_x, void* stream);
+
+/*
+ * Bytes of device workspace w4a8_linear needs for (M, K, N), or 0 if the
+ * shape breaks the rules.  The workspace holds the quantised activations,
+ * their scales and the split-K partial sums; its content need not be
+ * initialised and is scratch between calls.
+ */
+size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/*
+ * The layer: y[m, n] = bf16( s_x[m] * sum_k x_q[m,k] * W_hat[n,k] ), the
+ * sum accumulated in fp32 (ConvRot card, "Why this exists": the 4-bit
+ * weights are re-read on every token; "Format": the three scaling tiers).
+ *   x          [M, K] bf16 bit patterns (uint16), row-major.
+ *   packed     a buffer filled by w4a8_pack_layout for the same (N, K).
+ *   y          output [M, N] bf16 bit patterns (uint16), row-major.
+ *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
+ * M <= 16 runs the decode kernel (a weight-streaming GEMV); larger M runs
+ * the tensor-core GEMM.  Two calls sharing one workspace must be ordered on
+ * the GPU (same stream, or synchronised).
+ * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA.
+ */
+w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K,
+                        const void* packed, int64_t N, uint16_t* y,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The two halves of w4a8_linear, for callers that apply several layers of
+ * the same shape to one activation or that time the GEMM on its own.
+ *
+ * w4a8_linear_prepare: rotate and quantise x [M, K] (bf16 bits) into
+ *   `workspace`, laid out for a layer of N output rows (ConvRot card,
+ *   "Format": group-256 Hadamard rotation; W4A8 card, "Model Overview": int8
+ *   activations).
+ * w4a8_linear_run: y [M, N] = the layer applied to the activations the last
+ *   prepare on this workspace wrote.  It must be called with the same (M, K,
+ *   N) as that prepare, may be called any number of times after it (each run
+ *   leaves the workspace ready for another), and must be ordered after it on
+ *   the GPU.
+ * Errors: as w4a8_linear.
+ */
+w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N,
+                                void* workspace, size_t workspace_bytes, void* stream);
+w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
+                            uint16_t* y, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * Synchronise `stream`, then report and clear the device-side error word of
+ * the current device: W4A8_ERR_TIMEOUT if a bounded wait inside a kernel
+ * gave up since the last call (the affected outputs are then undefined),
+ * W4A8_ERR_CUDA if the synchronisation itself failed, else W4A8_OK.
+ */
+w4a8_status w4a8_get_device_error(void* stream);
+
+/* Static English description of a status code. */
+const char* w4a8_status_string(w4a8_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H_ */

@@ -27,5 +27,7 @@ def lib():
     """The CUDA library through its Python binding (GPU tests only)."""
     if not cuda_available():
         pytest.skip("no CUDA device")
+    import __graft_entry__
+    __graft_entry__.build()
     from w4a8_codebook_quantized_rotate_b200 import binding
     return binding

@@ -1,0 +1,86 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, it
+exports every function declared in include/w4a8.h, the size functions agree
+with the layout arithmetic, and bad arguments are refused before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    from w4a8_codebook_quantized_rotate_b200 import binding
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const char\*|size_t|w4a8_status)\s+(w4a8_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted([
+        "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
+        "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
+        "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_status_string", "w4a8_unpack_dequant"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_packed_bytes_layout_arithmetic(lib):
+    n, k = 17408, 5120
+    idx = n * k // 2
+    srel = n * k // 16
+    sch = -(-4 * n // 256) * 256
+    assert lib.w4a8_packed_bytes(n, k) == 256 + sch + idx + srel
+    assert lib.w4a8_packed_bytes(16, 256) == 256 + 256 + 16 * 128 + 16 * 16
+
+
+@pytest.mark.parametrize("n,k", [(0, 256), (8, 256), (24, 256), (16, 300), (16, 0), (16, 65536), (-16, 256)])
+def test_bad_weight_shapes_have_zero_size(lib, n, k):
+    assert lib.w4a8_packed_bytes(n, k) == 0
+    assert lib.w4a8_linear_workspace_bytes(1, k, n) == 0
+
+
+def test_workspace_sizes(lib):
+    assert lib.w4a8_linear_workspace_bytes(0, 256, 16) == 0
+    dec = lib.w4a8_linear_workspace_bytes(1, 5120, 17408)
+    pre = lib.w4a8_linear_workspace_bytes(4096, 5120, 17408)
+    assert dec > 5120 * 16 and pre >= 4096 * 5120 * 2 + 4096 * 4
+
+
+def test_null_and_shape_errors_before_launch(lib):
+    buf = ctypes.create_string_buffer(4096 + 16)
+    p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16   # 16-byte aligned host address
+    assert lib.w4a8_pack_layout(None, p, p, p, 16, 256, p, 4096, None) == 1
+    assert lib.w4a8_pack_layout(p, p, p, p, 16, 300, p, 4096, None) == 2
+    assert lib.w4a8_pack_layout(p + 1, p, p, p, 16, 256, p, 4096, None) == 3
+    assert lib.w4a8_pack_layout(p, p, p, p, 16, 256, p, 16, None) == 4
+    assert lib.w4a8_unpack_dequant(None, 16, 256, p, None) == 1
+    assert lib.w4a8_unpack_dequant(p, 15, 256, p, None) == 2
+    assert lib.w4a8_rotate_quant_act(p, 1, 255, p, p, None) == 2
+    assert lib.w4a8_rotate_quant_act(p, 0, 256, p, p, None) == 2
+    assert lib.w4a8_rotate_quant_act(p, 1, 256, p + 8, p, None) == 3
+    assert lib.w4a8_linear(p, 1, 256, p, 16, p, None, 0, None) == 1
+    assert lib.w4a8_linear(p, 1, 256, p, 17, p, p, 1 << 30, None) == 2
+    assert lib.w4a8_linear(p, 1, 256, p, 16, p, p, 16, None) == 4
+    assert lib.w4a8_linear_prepare(None, 1, 256, 16, p, 1 << 30, None) == 1
+    assert lib.w4a8_linear_prepare(p, 1, 256, 16, p + 4, 1 << 30, None) == 3
+    assert lib.w4a8_linear_run(1, 256, p, 16, p, p, 8, None) == 4
+    assert lib.w4a8_linear_run(1, 512, p, 16, None, p, 1 << 30, None) == 1
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.w4a8_status_string(s)
+    assert b"unknown" in lib.w4a8_status_string(99)

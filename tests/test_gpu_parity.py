@@ -1,0 +1,261 @@
+"""Parity of the CUDA library (through its C ABI) against the CPU oracle.
+
+Bars (the layer's stated tolerances):
+  * dequantisation and layout: bit-exact;
+  * int8 activations: at most 1 LSB apart, on at most 1e-4 of the elements;
+  * linear output (bf16) against the unrounded fp64 oracle: relative L2
+    error <= 2e-3 and, per token m, max |error| <= 1e-2 * ||x_m||_2 * max|W_hat|;
+  * integer-valued special cases: exact.
+Shapes span several tiles and ragged tails (odd tile counts, token counts
+that are not multiples of 8 or 256) and the full workload shapes (sampled
+outputs, computed one by one by the oracle).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 2e-3
+MAX_ABS_FACTOR = 1e-2
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def bf16(bits):
+    return dev(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def pack(lib, q):
+    return lib.pack_layout(dev(q["packed"]), dev(q["s_rel"]), dev(q["s_ch"]), dev(q["cb"]))
+
+
+def converted(n, k, seed):
+    w = synth.weights(n, k, synth.rng_for(seed, 0, "weight"))
+    return O.convert_weight(w)
+
+
+def check_linear(y_gpu, y_ref, x, w_maxabs):
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    err = y_gpu - y_ref
+    rel = np.linalg.norm(err) / np.linalg.norm(y_ref)
+    assert rel <= REL_L2, f"relative L2 error {rel:.3e}"
+    bound = MAX_ABS_FACTOR * np.linalg.norm(np.asarray(x, dtype=np.float64), axis=1) * w_maxabs
+    worst = np.max(np.abs(err), axis=1)
+    assert np.all(worst <= bound), f"max abs error {worst.max():.3e} > bound {bound.min():.3e}"
+    return rel
+
+
+def run_linear(lib, x_bits, packed, n):
+    return lib.linear(bf16(x_bits), packed, n).float().cpu().numpy()
+
+
+# ------------------------------------------------------------------ dequant / layout
+
+@pytest.mark.parametrize("n,k,seed", [(256, 512, 0), (592, 768, 1), (16, 256, 2)])
+def test_dequant_bit_exact(lib, n, k, seed):
+    c = converted(n, k, seed)
+    got = lib.unpack_dequant(pack(lib, c), n, k).cpu().numpy()
+    ref = O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_dequant_edge_scales_bit_exact(lib):
+    """Subnormal and zero e4m3 scales, zero rows and extreme levels."""
+    rng = np.random.default_rng(20)
+    n, k = 64, 512
+    q = synth.quantized_format(n, k, rng)
+    q["s_rel"][:, ::3] = rng.integers(0, 8, size=q["s_rel"][:, ::3].shape)  # subnormals and zero
+    q["s_rel"][5] = 0
+    q["s_ch"][7] = 0.0
+    q["s_ch"][9] = np.float32(1e-30)
+    q["cb"] = np.array([-3.0e-8, *np.linspace(-1, 1, 14), 7.5], dtype=np.float32)
+    got = lib.unpack_dequant(pack(lib, q), n, k).cpu().numpy()
+    ref = O.dequant_packed(q["packed"], q["s_rel"], q["s_ch"], q["cb"])
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_dequant_full_size_sampled_rows(lib):
+    n, k = 17408, 5120
+    q = synth.quantized_format(n, k, synth.rng_for(1, 0, "qfmt"))
+    got = lib.unpack_dequant(pack(lib, q), n, k)
+    rows = np.sort(synth.rng_for(1, 0, "sample").choice(n, 96, replace=False))
+    ref = O.dequant_packed(q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=rows)
+    assert np.array_equal(got[torch.from_numpy(rows).cuda()].cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+# ------------------------------------------------------------------ activations
+
+def flips_ok(q_gpu, q_ref):
+    d = np.abs(q_gpu.astype(np.int32) - q_ref.astype(np.int32))
+    assert d.max() <= 1, f"int8 codes differ by {d.max()}"
+    allowed = math.ceil(1e-4 * d.size)
+    assert np.count_nonzero(d) <= allowed, f"{np.count_nonzero(d)} flips > {allowed}"
+
+
+@pytest.mark.parametrize("m,k,outl", [(4, 512, 2), (37, 768, 8), (1, 5120, 51), (16, 17408, 174), (64, 17408, 174)])
+def test_rotate_quant_matches_oracle(lib, m, k, outl):
+    bits, x, _ = synth.activations(m, k, synth.rng_for(7, m, "act"), outl)
+    xq, sx = lib.rotate_quant_act(bf16(bits))
+    q_ref, s_ref, _ = O.quantize_activations(x)
+    sx = sx.cpu().numpy()
+    assert np.all(np.abs(sx.view(np.int32) - s_ref.view(np.int32)) <= 1)   # within 1 ulp
+    flips_ok(xq.cpu().numpy(), q_ref)
+
+
+def test_rotate_quant_special_rows(lib):
+    k = 512
+    x = np.zeros((3, k), dtype=np.float32)
+    x[1, :256] = scipy.linalg.hadamard(256)[5] * (3.0 / 16.0)   # rotates to a spike of 3 at k = 5
+    x[2, 300] = -2.0                                             # rotates to a flat block
+    bits = synth.f32_to_bf16_bits(x)
+    xq, sx = lib.rotate_quant_act(bf16(bits))
+    q_ref, s_ref, _ = O.quantize_activations(x)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy(), s_ref)
+    assert sx[0].item() == 0.0
+
+
+# ------------------------------------------------------------------ linear
+
+@pytest.fixture(scope="module")
+def layer592(lib):
+    c = converted(592, 768, 3)          # 37 tiles of 16 rows: an odd tile count
+    return c, pack(lib, c), float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 5, 8, 9, 13, 16])
+def test_linear_decode_matches_oracle(lib, layer592, m):
+    c, packed, wmax = layer592
+    bits, x, _ = synth.activations(m, 768, synth.rng_for(4, m, "act"), 8)
+    y = run_linear(lib, bits, packed, 592)
+    check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+@pytest.mark.parametrize("m", [17, 64, 255, 256, 300])
+def test_linear_prefill_matches_oracle(lib, layer592, m):
+    c, packed, wmax = layer592
+    bits, x, _ = synth.activations(m, 768, synth.rng_for(5, m, "act"), 8)
+    y = run_linear(lib, bits, packed, 592)
+    check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+@pytest.mark.parametrize("m,n,k", [(4, 256, 512), (513, 256, 512), (1, 16, 256), (40, 16, 256), (3, 4096, 1024)])
+def test_linear_small_shapes(lib, m, n, k):
+    c = converted(n, k, 6)
+    wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+    bits, x, _ = synth.activations(m, k, synth.rng_for(6, m, "act"), 2)
+    y = run_linear(lib, bits, pack(lib, c), n)
+    check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+def integer_case(m, n, k, seed):
+    """Integer codebook, unit scales, and activations whose rotation is a
+    spike per 256-block: every sum is a small integer, so y is exact."""
+    rng = np.random.default_rng(seed)
+    nb = k // 256
+    cb = np.arange(-8, 8).astype(np.float32)
+    idx = rng.integers(0, 16, size=(n, k)).astype(np.uint8)
+    hs = scipy.linalg.hadamard(256)
+    x = np.zeros((m, k), dtype=np.float32)
+    expect = np.zeros((m, n))
+    for r in range(m):
+        pos = rng.integers(0, 256, size=nb)
+        qv = rng.integers(-4, 5, size=nb)
+        qv[0] = 127                        # sets s_x = 1 exactly
+        idx[:, pos[0]] = 8                 # level 0.0 under the 127 spike, for every row
+        for b in range(nb):
+            x[r, 256 * b: 256 * (b + 1)] = hs[pos[b]] * (qv[b] / 16.0)
+        # filled in after idx is final, below
+        expect[r] = 0
+    # expected values from the final index table
+    for r in range(m):
+        xr = O.rotate_blocks(x[r:r + 1])[0]
+        nz = np.nonzero(np.rint(xr))[0]
+        expect[r] = (np.rint(xr[nz])[None, :] * cb[idx[:, nz].astype(np.int64)]).sum(axis=1)
+    q = {"packed": O.pack_nibbles(idx), "s_rel": np.full((n, k // 16), 0x38, np.uint8),
+         "s_ch": np.ones(n, np.float32), "cb": cb}
+    return q, x, expect
+
+
+@pytest.mark.parametrize("m", [1, 4, 16, 300])
+def test_linear_exact_integer_case(lib, m):
+    n, k = 272, 768
+    q, x, expect = integer_case(m, n, k, 30 + m)
+    assert np.abs(expect).max() <= 256      # bf16 represents these exactly
+    y = run_linear(lib, synth.f32_to_bf16_bits(x), pack(lib, q), n)
+    assert np.array_equal(y.astype(np.float64), expect)
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 5120, 17408), (1, 17408, 5120), (4, 17408, 5120), (16, 17408, 5120),
+                                   (4096, 5120, 17408), (8192, 17408, 5120)])
+def test_linear_full_size_sampled(lib, m, k, n):
+    """Workload shapes in the launch configuration the benchmark times; the
+    oracle computes a sample of outputs (tokens x output rows)."""
+    q = synth.quantized_format(n, k, synth.rng_for(11, n, "qfmt"))
+    bits, x, _ = synth.activations(m, k, synth.rng_for(11, m, "act"), max(1, k // 100))
+    y = lib.linear(bf16(bits), pack(lib, q), n)
+    srng = synth.rng_for(11, m, "sample")
+    toks = np.sort(srng.choice(m, min(m, 24), replace=False))
+    rows = np.sort(srng.choice(n, 128, replace=False))
+    y_s = y[torch.from_numpy(toks).cuda()][:, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    ref = O.linear_packed(x[toks], q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=rows)
+    wmax = float(np.abs(O.dequant_packed(q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=rows)).max())
+    check_linear(y_s, ref, x[toks], wmax)
+
+
+@pytest.mark.parametrize("m", [1, 16, 300])
+def test_linear_deterministic_and_workspace_reuse(lib, layer592, m):
+    c, packed, _ = layer592
+    bits, _, _ = synth.activations(m, 768, synth.rng_for(8, m, "act"), 8)
+    xt = bf16(bits)
+    ws = torch.empty(lib.linear_workspace_bytes(4096, 768, 592) + 4096, dtype=torch.uint8, device="cuda")
+    a = lib.linear(xt, packed, 592, workspace=ws).clone()
+    # a different shape through the same workspace in between
+    other, _, _ = synth.activations(5, 768, synth.rng_for(8, 99, "act"), 8)
+    lib.linear(bf16(other), packed, 592, workspace=ws)
+    b = lib.linear(xt, packed, 592, workspace=ws)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_binding_refuses_bad_arguments(lib, layer592):
+    c, packed, _ = layer592
+    with pytest.raises(ValueError):
+        lib.linear(torch.zeros(2, 768, device="cuda"), packed, 592)           # fp32 input
+    with pytest.raises(Exception):
+        lib.linear(torch.zeros(2, 700, dtype=torch.bfloat16, device="cuda"), packed, 592)   # K % 256
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception):
+        lib.linear(torch.zeros(2, 768, dtype=torch.bfloat16, device="cuda"), packed, 592, workspace=small)
+
+
+def test_no_device_error_recorded(lib):
+    assert lib.get_device_error() == 0
+
+
+@pytest.mark.parametrize("m", [1, 4, 300])
+def test_prepare_once_run_several_layers(lib, m):
+    """One prepared activation, several layers of the same shape, each run
+    equal to the fused call and to the oracle."""
+    n, k = 592, 768
+    layers = [converted(n, k, 40 + i) for i in range(3)]
+    bits, x, _ = synth.activations(m, k, synth.rng_for(9, m, "act"), 8)
+    xt = bf16(bits)
+    ws = torch.empty(lib.linear_workspace_bytes(m, k, n), dtype=torch.uint8, device="cuda")
+    lib.linear_prepare(xt, n, ws)
+    for c in layers:
+        packed = pack(lib, c)
+        y_run = lib.linear_run(m, k, packed, n, ws)
+        y_ref = lib.linear(xt, packed, n)
+        assert torch.equal(y_run.view(torch.int16), y_ref.view(torch.int16))
+        wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+        check_linear(y_run.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)

@@ -1,0 +1,143 @@
+// Activation rotation and per-token int8 quantisation.
+//
+// x_rot[m, 256 b + j] = (1/16) sum_i x[m, 256 b + i] H_256[i, j]  (Sylvester H)
+// s_x[m] = max_k |x_rot[m, k]| / 127,  q = clamp(rint(x_rot / s_x), -127, 127)
+//
+// "Qwen3.8-27B-AEON-ULTIMATE-UNCENSORED-BF16 -- W4A8 ConvRot for ComfyUI"
+// model card, section "Format" (group-wise Hadamard rotation, group 256);
+// "Qwen3.8-27B-W4A8" model card, section "Model Overview" (int8
+// activations).  The weights were rotated by the same orthonormal H_256/16,
+// so x_rot . W_rot = x . W.
+//
+// One CTA per token.  Each warp transforms whole 256-blocks: a lane holds 8
+// consecutive values, the three butterfly stages inside a lane run in
+// registers and the five across lanes use shuffles.  The rotated row is
+// staged in shared memory until the row maximum is known.
+#pragma once
+
+#include "common.cuh"
+
+namespace w4a8 {
+
+enum ActOut : int {
+  kActI8Row = 0,    // int8 [M, K] row-major (the C ABI's rotate-quant call)
+  kActF16Row = 1,   // fp16 [M, K] row-major, the tensor-core GEMM's operand
+  kActF16Frag = 2,  // fp16 in mma.sync B-fragment order, the decode kernel's operand
+};
+
+constexpr int kActThreads = 256;
+
+// Index (in half2 units) of element (m, k) in the decode B-fragment layout:
+// [chunk][n8 block j][lane 32][8 half2], lane = 4 (m % 8) + t, half2
+// register 2 s + w holds k = 64 chunk + 16 s + 2 t + 8 w and k + 1.
+__host__ __device__ inline int64_t frag_half2_index(int64_t m, int64_t k, int nb) {
+  const int64_t c = k >> 6;
+  const int s = int(k >> 4) & 3, w = int(k >> 3) & 1, t = int(k >> 1) & 3;
+  const int64_t j = m >> 3;
+  const int g = int(m & 7);
+  return (((c * nb + j) * 32 + 4 * g + t) * 8) + 2 * s + w;
+}
+
+__device__ __forceinline__ void fwht8_in_lane(float (&v)[8]) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+}
+
+template <int OUT>
+__global__ void __launch_bounds__(kActThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                                  void* __restrict__ out, float* __restrict__ s_x,
+                                                                  int nb, unsigned* __restrict__ zero_words,
+                                                                  int zero_count) {
+  extern __shared__ float xr[];  // [K] rotated row
+  __shared__ float warp_max[kActThreads / 32];
+  // Later kernels may start their weight streaming now; they wait for this
+  // grid's completion before reading anything it writes.
+  pdl_launch_dependents();
+  const int m = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (zero_words && m == 0) {
+    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_words[i] = 0u;
+  }
+  const int nblocks = K / kRotBlock;
+  float amax = 0.f;
+  for (int b = warp; b < nblocks; b += kActThreads / 32) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(x + int64_t(m) * K + b * kRotBlock + lane * 8);
+    const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(wds[i] << 16);
+      v[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+    }
+    fwht8_in_lane(v);
+#pragma unroll
+    for (int bit = 1; bit < 32; bit <<= 1) {
+      const bool upper = (lane & bit) != 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float p = __shfl_xor_sync(0xffffffffu, v[i], bit);
+        v[i] = upper ? (p - v[i]) : (v[i] + p);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] *= 0.0625f;  // 1/16, exact
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+    float4* dst = reinterpret_cast<float4*>(xr + b * kRotBlock + lane * 8);
+    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int i = 1; i < kActThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (threadIdx.x == 0) s_x[m] = s;
+  // Quantise 8 consecutive values per thread per step.
+  for (int k0 = threadIdx.x * 8; k0 < K; k0 += kActThreads * 8) {
+    const float4 a = *reinterpret_cast<const float4*>(xr + k0);
+    const float4 c = *reinterpret_cast<const float4*>(xr + k0 + 4);
+    const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q[i] = s > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -127.f), 127.f) : 0.f;
+    }
+    if constexpr (OUT == kActI8Row) {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo |= (uint32_t(int(q[i])) & 0xFFu) << (8 * i);
+        hi |= (uint32_t(int(q[i + 4])) & 0xFFu) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + int64_t(m) * K + k0) = make_uint2(lo, hi);
+    } else if constexpr (OUT == kActF16Row) {
+      __half2 h[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
+      *reinterpret_cast<uint4*>(static_cast<__half*>(out) + int64_t(m) * K + k0) =
+          *reinterpret_cast<uint4*>(h);
+    } else {
+      __half2* o = static_cast<__half2*>(out);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[frag_half2_index(m, k0 + 2 * i, nb)] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
+      }
+    }
+  }
+}
+
+}  // namespace w4a8

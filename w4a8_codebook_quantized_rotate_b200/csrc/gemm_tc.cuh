@@ -1,0 +1,296 @@
+// Prefill kernel (M > 16): tensor-core GEMM on tcgen05 with the codebook
+// expansion fused into the operand path.
+//
+// The product is computed transposed, D^T[n, m] = sum_k W'[n, k] x_q[m, k],
+// so that the expanded weight is the MMA's A operand, which tcgen05 can read
+// from tensor memory:
+//   * 4 expansion warps turn a 128-row x 64-k block of packed indices into
+//     fp16 W' = fp16(fp16(cb[idx]) * s_rel) and store it straight into TMEM
+//     with tcgen05.st -- the expansion never touches shared-memory
+//     bandwidth, which the B operand and the TMA engine need;
+//   * a TMA warp loads x_q (fp16, integer-valued, exact) tiles of 256 tokens
+//     x 64 k into 128-byte-swizzled shared memory (no multicast);
+//   * one thread issues tcgen05.mma kind::f16 (M = 128 weight rows, N = 256
+//     tokens, K = 16) into an fp32 accumulator in TMEM;
+//   * the expansion warps then read the accumulator back (tcgen05.ld), scale
+//     by s_ch[n] s_x[m] in fp32 and store y in bf16.
+// "Qwen3.8-27B-AEON-ULTIMATE-UNCENSORED-BF16 -- W4A8 ConvRot for ComfyUI"
+// model card, "Why this exists" and "Format": the layer runs a tensor-core
+// GEMM with a codebook dequantisation step on top.  The pages' int8 operand
+// cannot hold the three-tier weight within the output tolerance, so the
+// operand here is fp16 (the accumulation is fp32 either way).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace w4a8 {
+
+constexpr int kTcRows = 128;      // weight rows per tile (TMEM lanes, MMA M)
+constexpr int kTcTokens = 256;    // tokens per tile (MMA N)
+constexpr int kTcBK = 64;         // k per pipeline stage
+constexpr int kTcStagesB = 3;     // x_q stages in shared memory
+constexpr int kTcStagesA = 4;     // expanded-weight stages in TMEM
+constexpr int kTcThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 expansion + epilogue
+constexpr uint32_t kTcStageBBytes = kTcTokens * kTcBK * 2;  // 32 KiB
+constexpr uint32_t kTcTmemCols = 512;
+constexpr uint32_t kTcAccCol = 0;     // accumulator: columns [0, 256)
+constexpr uint32_t kTcACol = 256;     // A stages: columns [256, 384)
+// dynamic shared memory: [barriers | pad to the next 64 KiB boundary] [LUT 64 KiB] [B stages]
+constexpr size_t kTcSmemBytes = 1024 + 65536 + 65536 + size_t(kTcStagesB) * kTcStageBBytes;
+
+struct TcParams {
+  const uint8_t* idx;
+  const uint8_t* srel;
+  const float* sch;
+  const float* cb;
+  const float* s_x;
+  uint16_t* y;
+  unsigned* err;
+  int M, N, K, C, T;
+};
+
+struct TcShared {
+  uint64_t b_full[kTcStagesB];
+  uint64_t b_empty[kTcStagesB];
+  uint64_t a_full[kTcStagesA];
+  uint64_t a_empty[kTcStagesA];
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+// Instruction descriptor, kind::f16: fp16 A and B, fp32 D, both K-major,
+// M = 128 (bits 24..28 hold M >> 4), N = 256 (bits 17..22 hold N >> 3).
+constexpr uint32_t kTcIdesc = (1u << 4) | (uint32_t(kTcTokens >> 3) << 17) | (uint32_t(kTcRows >> 4) << 24);
+
+// Shared-memory descriptor of a K-major tile with 128-byte swizzling: rows
+// of 128 bytes, 8-row groups 1024 bytes apart (SBO), LBO unused (1), format
+// version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+  return uint64_t((smem_addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Bounded wait that also gives up once another role has aborted.  About a
+// million polls, each of which may suspend the thread briefly: on the order
+// of a second before the kernel records a timeout and unwinds.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, TcShared* sh, unsigned* err) {
+  for (uint32_t i = 0; i < (1u << 20); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 1023u && sh->abort) return false;
+  }
+  sh->abort = 1;
+  record_error(err, kErrTimeout);
+  return false;
+}
+
+struct ExpStage {
+  uint4 seg[4];  // the four 16-byte lane segments holding this row's index bytes
+  uint2 sr;      // group-scale bytes of rows (g, g+8) for the chunk's 4 groups
+};
+
+__device__ __forceinline__ void exp_load(ExpStage& e, const TcParams& p, int tile, int kb, int g, bool valid) {
+  if (valid && kb < p.C) {
+    const size_t blk = size_t(tile) * p.C + kb;
+    const uint8_t* src = p.idx + blk * kChunkIdxBytes + size_t(4 * g) * 16;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) e.seg[t] = __ldg(reinterpret_cast<const uint4*>(src) + t);
+    e.sr = __ldg(reinterpret_cast<const uint2*>(p.srel + blk * kChunkSrelBytes + g * 8));
+  } else {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) e.seg[t] = make_uint4(0, 0, 0, 0);
+    e.sr = make_uint2(0, 0);
+  }
+}
+
+// Expand one row's 64 k of one chunk into 32 fp16 pairs (TMEM column
+// 8 s + b holds k = 16 s + 2 b, 2 b + 1 of the chunk).
+__device__ __forceinline__ void exp_compute(const ExpStage& e, uint32_t lut_lane, int h, uint32_t (&out)[32]) {
+  const uint32_t sel_lo = 0x7604u | (uint32_t(h) << 4);        // byte h of a word: (row, b = t)
+  const uint32_t sel_hi = 0x7604u | (uint32_t(h + 2) << 4);    // byte h+2: (row, b = t + 4)
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t codes = (s < 2 ? e.sr.x : e.sr.y) >> (16 * (s & 1) + 8 * h);
+    __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(codes & 0xFFu), __NV_E4M3);
+    const __half sh = *reinterpret_cast<__half*>(&hr);
+    const __half2 sc = __halves2half2(sh, sh);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t word = s == 0 ? e.seg[t].x : s == 1 ? e.seg[t].y : s == 2 ? e.seg[t].z : e.seg[t].w;
+      uint32_t lo = lds_u32(prmt(word, lut_lane, sel_lo));
+      uint32_t hi = lds_u32(prmt(word, lut_lane, sel_hi));
+      __half2 vlo = __hmul2(*reinterpret_cast<__half2*>(&lo), sc);
+      __half2 vhi = __hmul2(*reinterpret_cast<__half2*>(&hi), sc);
+      out[8 * s + t] = *reinterpret_cast<uint32_t*>(&vlo);
+      out[8 * s + t + 4] = *reinterpret_cast<uint32_t*>(&vhi);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t tc_smem[];
+  TcShared* sh = reinterpret_cast<TcShared*>(tc_smem);
+  const uint32_t base = smem_u32(tc_smem);
+  // 64 KiB aligned (bits 8..15 zero), past the barrier block
+  const uint32_t lut = (base + uint32_t(sizeof(TcShared)) + 0xFFFFu) & ~0xFFFFu;
+  const uint32_t bstage0 = lut + 65536u;  // 1024-byte aligned
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTcRows;
+  const int m0 = blockIdx.y * kTcTokens;
+  const int KB = p.C;  // k blocks of 64
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStagesB; ++s) {
+      mbar_init(&sh->b_full[s], 1);
+      mbar_init(&sh->b_empty[s], 1);
+    }
+    for (int s = 0; s < kTcStagesA; ++s) {
+      mbar_init(&sh->a_full[s], 128);
+      mbar_init(&sh->a_empty[s], 1);
+    }
+    mbar_init(&sh->acc_full, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, kTcTmemCols);
+    tmem_relinquish();
+  }
+  // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
+  for (int e = threadIdx.x; e < 256 * 32; e += kTcThreads) {
+    const int b = e >> 5;
+    const __half2 h = __floats2half2_rn(p.cb[b & 15], p.cb[b >> 4]);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(e & 31) * 4u),
+                 "r"(*reinterpret_cast<const uint32_t*>(&h)));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer: x_q tiles
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_x);
+      pdl_wait();  // x_q and s_x are written by the previous kernel
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % kTcStagesB;
+        if (!tc_wait(&sh->b_empty[s], ((kb / kTcStagesB) & 1) ^ 1, sh, p.err)) break;
+        mbar_arrive_expect_tx(&sh->b_full[s], kTcStageBBytes);
+        tma_load_2d(bstage0 + uint32_t(s) * kTcStageBBytes, &tmap_x, &sh->b_full[s], kb * kTcBK, m0);
+        ++issued;
+      }
+      if (sh->abort) {  // let copies already in flight land before the CTA exits
+        for (int i = issued > kTcStagesB ? issued - kTcStagesB : 0; i < issued; ++i)
+          mbar_wait_bounded(&sh->b_full[i % kTcStagesB], (i / kTcStagesB) & 1, p.err, 1u << 20);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int sa = kb % kTcStagesA, sb = kb % kTcStagesB;
+        ok = tc_wait(&sh->a_full[sa], (kb / kTcStagesA) & 1, sh, p.err) &&
+             tc_wait(&sh->b_full[sb], (kb / kTcStagesB) & 1, sh, p.err);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < kTcBK / 16; ++j) {
+          const uint32_t a = tmem + kTcACol + uint32_t(sa) * 32u + uint32_t(j) * 8u;
+          const uint64_t bd = sw128_desc(bstage0 + uint32_t(sb) * kTcStageBBytes + uint32_t(j) * 32u);
+          tc_mma_ts_f16(tmem + kTcAccCol, a, bd, kTcIdesc, (kb | j) != 0 ? 1u : 0u);
+        }
+        tc_commit(&sh->a_empty[sa]);
+        tc_commit(&sh->b_empty[sb]);
+      }
+      if (ok) {
+        tc_commit(&sh->acc_full);
+      } else {  // wait for the MMAs already issued before the TMEM is freed
+        tc_commit(&sh->drain);
+        mbar_wait_bounded(&sh->drain, 0, p.err, 1u << 20);
+      }
+    }
+  } else {
+    // ------------------------------------------------ expansion, then epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = 32 * q + lane;
+    const int n = n0 + r;
+    const bool valid = n < p.N;
+    const int tile = n >> 4, g = n & 7, h = (n >> 3) & 1;
+    const uint32_t lut_lane = lut + uint32_t(lane) * 4u;
+    const uint32_t trow = uint32_t(32 * q) << 16;
+    constexpr int PF = 4;
+    ExpStage es[PF];
+#pragma unroll
+    for (int i = 0; i < PF; ++i) exp_load(es[i], p, tile, i, g, valid);
+    bool ok = true;
+    for (int kb0 = 0; kb0 < KB && ok; kb0 += PF) {
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        const int kb = kb0 + i;
+        if (kb < KB && ok) {
+          const int sa = kb % kTcStagesA;
+          uint32_t v[32];
+          exp_compute(es[i], lut_lane, h, v);
+          if (!valid) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = 0u;
+          }
+          exp_load(es[i], p, tile, kb + PF, g, valid);
+          // lane 0 polls; the verdict is made warp-uniform before the
+          // .sync.aligned TMEM store
+          int w_ok = lane == 0 ? int(tc_wait(&sh->a_empty[sa], ((kb / kTcStagesA) & 1) ^ 1, sh, p.err)) : 0;
+          ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+          if (ok) {
+            tc_fence_after();
+            tmem_st_32x32b_x32(tmem + trow + kTcACol + uint32_t(sa) * 32u, v);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sh->a_full[sa]);
+          }
+        }
+      }
+    }
+    int acc_ok = (ok && lane == 0) ? int(tc_wait(&sh->acc_full, 0, sh, p.err)) : 0;
+    if (__shfl_sync(0xffffffffu, acc_ok, 0) != 0) {
+      tc_fence_after();
+      pdl_wait();  // s_x comes from the previous kernel
+      const float sch = valid ? p.sch[n] : 0.f;
+#pragma unroll 1
+      for (int ci = 0; ci < kTcTokens / 32; ++ci) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + trow + kTcAccCol + uint32_t(ci) * 32u, v);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m0 + ci * 32 + j;
+            if (m < p.M) {
+              const float val = __uint_as_float(v[j]) * sch * p.s_x[m];
+              p.y[size_t(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTcTmemCols);
+}
+
+}  // namespace w4a8

@@ -1,0 +1,359 @@
+// C ABI of the W4A8 ConvRot linear layer: argument checks, per-device set-up
+// and kernel launches.  The declarations, with argument meaning, layout,
+// ownership and error behaviour, are in include/w4a8.h.
+#include <mutex>
+
+#include "w4a8.h"
+
+#include "act.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+
+namespace w4a8 {
+
+// Device-side error word (bit flags, kErrTimeout); read and cleared by
+// w4a8_get_device_error.
+__device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  bool arch_ok = false;
+  int sms = 0;
+  unsigned* err = nullptr;
+};
+
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool weight_shape_ok(int64_t N, int64_t K) {
+  return N > 0 && N % kTileRows == 0 && N <= (int64_t(1) << 24) && K > 0 && K % kRotBlock == 0 && K <= kMaxK;
+}
+
+bool act_shape_ok(int64_t M, int64_t K) {
+  return M > 0 && M <= (int64_t(1) << 24) && K > 0 && K % kRotBlock == 0 && K <= kMaxK;
+}
+
+template <typename Kern>
+cudaError_t allow_smem(Kern k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+}
+
+// Per-device state: architecture check, SM count, error-word address and
+// the shared-memory opt-ins of the large kernels.  Done once per device.
+w4a8_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& d = g_devices[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return W4A8_ERR_CUDA;
+    d.arch_ok = (major == 10 && minor == 0);
+    d.sms = sms;
+    if (d.arch_ok) {
+      void* sym = nullptr;
+      if (cudaGetSymbolAddress(&sym, g_error_word) != cudaSuccess) return W4A8_ERR_CUDA;
+      d.err = static_cast<unsigned*>(sym);
+      if (allow_smem(rotate_quant_kernel<kActI8Row>, size_t(kMaxK) * 4) != cudaSuccess ||
+          allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
+          allow_smem(rotate_quant_kernel<kActF16Frag>, size_t(kMaxK) * 4) != cudaSuccess ||
+          allow_smem(decode_kernel<1, 4, true>, kDecSmemBytes) != cudaSuccess ||
+          allow_smem(decode_kernel<1, 4, false>, kDecSmemBytes) != cudaSuccess ||
+          allow_smem(decode_kernel<2, 2, false>, kDecSmemBytes) != cudaSuccess ||
+          allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
+        return W4A8_ERR_CUDA;
+    }
+    d.ready = true;
+  }
+  if (!d.arch_ok) return W4A8_ERR_ARCH;
+  *out = &d;
+  return W4A8_OK;
+}
+
+w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA; }
+
+// ------------------------------------------------------------------ linear workspace
+
+constexpr int kDecodeMaxM = 16;
+
+struct LinearPlan {
+  bool decode;
+  int nb;          // decode: token blocks of 8
+  size_t off_sx, off_xq, off_cnt, off_slots, total;
+  int T, P, C;
+};
+
+LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
+  LinearPlan L{};
+  L.decode = M <= kDecodeMaxM;
+  L.T = int(N / kTileRows);
+  L.C = int(K / kChunkK);
+  L.P = (L.T + kDecTG - 1) / kDecTG;
+  if (L.decode) {
+    L.nb = int((M + 7) / 8);
+    L.off_sx = 0;
+    L.off_xq = 256;
+    L.off_cnt = round_up(L.off_xq + size_t(K) * L.nb * 16, 256);
+    L.off_slots = round_up(L.off_cnt + size_t(L.P) * 4, 256);
+    L.total = round_up(L.off_slots + size_t(2) * kDecMaxWarps * dec_slot_floats(L.nb) * 4, 256);
+  } else {
+    L.nb = 0;
+    L.off_sx = 0;
+    L.off_xq = round_up(size_t(M) * 4, 256);
+    L.off_cnt = L.off_slots = 0;
+    L.total = round_up(L.off_xq + size_t(M) * K * 2, 256);
+  }
+  return L;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace
+}  // namespace w4a8
+
+using namespace w4a8;
+
+extern "C" {
+
+size_t w4a8_packed_bytes(int64_t N, int64_t K) {
+  if (!weight_shape_ok(N, K)) return 0;
+  return packed_layout(N, K).total;
+}
+
+w4a8_status w4a8_pack_layout(const uint8_t* idx, const uint8_t* s_rel, const float* s_channel,
+                             const float* codebook, int64_t N, int64_t K, void* packed, size_t packed_bytes,
+                             void* stream) {
+  if (!idx || !s_rel || !s_channel || !codebook || !packed) return W4A8_ERR_NULL;
+  if (!weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(idx) || !aligned16(s_rel) || !aligned16(s_channel) || !aligned16(codebook) || !aligned16(packed))
+    return W4A8_ERR_ALIGN;
+  const PackedLayout L = packed_layout(N, K);
+  if (packed_bytes < L.total) return W4A8_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(packed);
+  const int64_t threads = L.tiles * L.chunks * 32;
+  pack_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(idx, s_rel, N, K, base + L.off_idx,
+                                                              base + L.off_srel);
+  copy_scales_kernel<<<unsigned((N + 255) / 256), 256, 0, s>>>(s_channel, codebook, N,
+                                                                reinterpret_cast<float*>(base + L.off_sch),
+                                                                reinterpret_cast<float*>(base + L.off_cb));
+  return launch_status();
+}
+
+w4a8_status w4a8_unpack_dequant(const void* packed, int64_t N, int64_t K, float* w_hat, void* stream) {
+  if (!packed || !w_hat) return W4A8_ERR_NULL;
+  if (!weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(w_hat)) return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  const PackedLayout L = packed_layout(N, K);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  const int64_t threads = L.tiles * L.chunks * 32;
+  dequant_kernel<<<unsigned((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      base + L.off_idx, base + L.off_srel, reinterpret_cast<const float*>(base + L.off_sch),
+      reinterpret_cast<const float*>(base + L.off_cb), N, K, w_hat);
+  return launch_status();
+}
+
+w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* x_q, float* s_x,
+                                  void* stream) {
+  if (!x || !x_q || !s_x) return W4A8_ERR_NULL;
+  if (!act_shape_ok(M, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(x_q) || !aligned16(s_x)) return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  rotate_quant_kernel<kActI8Row><<<unsigned(M), kActThreads, size_t(K) * 4, static_cast<cudaStream_t>(stream)>>>(
+      x, int(M), int(K), x_q, s_x, 0, nullptr, 0);
+  return launch_status();
+}
+
+size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (!act_shape_ok(M, K) || !weight_shape_ok(N, K)) return 0;
+  return linear_plan(M, K, N).total;
+}
+
+static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* workspace, size_t workspace_bytes,
+                                 LinearPlan* plan, DeviceState** d) {
+  if (!workspace) return W4A8_ERR_NULL;
+  if (!act_shape_ok(M, K) || !weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+  *plan = linear_plan(M, K, N);
+  if (workspace_bytes < plan->total) return W4A8_ERR_WORKSPACE;
+  return device_state(d);
+}
+
+w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!x) return W4A8_ERR_NULL;
+  if (!aligned16(x)) return W4A8_ERR_ALIGN;
+  LinearPlan plan;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = linear_checks(M, K, N, workspace, workspace_bytes, &plan, &d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(ws + plan.off_sx);
+  if (plan.decode) {
+    rotate_quant_kernel<kActF16Frag><<<unsigned(M), kActThreads, size_t(K) * 4, s>>>(
+        x, int(M), int(K), ws + plan.off_xq, s_x, plan.nb, reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P);
+  } else {
+    rotate_quant_kernel<kActF16Row><<<unsigned(M), kActThreads, size_t(K) * 4, s>>>(
+        x, int(M), int(K), ws + plan.off_xq, s_x, 0, nullptr, 0);
+  }
+  return launch_status();
+}
+
+w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N, uint16_t* y, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!packed || !y) return W4A8_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(y)) return W4A8_ERR_ALIGN;
+  LinearPlan plan;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = linear_checks(M, K, N, workspace, workspace_bytes, &plan, &d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const PackedLayout L = packed_layout(N, K);
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(ws + plan.off_sx);
+
+  if (plan.decode) {
+    DecodeParams p;
+    p.idx = pk + L.off_idx;
+    p.srel = pk + L.off_srel;
+    p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
+    p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
+    p.xfrag = reinterpret_cast<const uint4*>(ws + plan.off_xq);
+    p.s_x = s_x;
+    p.y = y;
+    p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
+    p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
+    p.err = d->err;
+    p.M = int(M);
+    p.N = int(N);
+    p.C = plan.C;
+    p.T = plan.T;
+    p.P = plan.P;
+    p.U = plan.P * plan.C;
+    const int warps_avail = (d->sms < 148 ? d->sms : 148) * kDecWarps;
+    p.W = p.U < warps_avail ? p.U : warps_avail;
+    const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
+    cudaError_t e;
+    if (plan.nb == 1 && M == 1)
+      e = launch_pdl(decode_kernel<1, 4, true>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+    else if (plan.nb == 1)
+      e = launch_pdl(decode_kernel<1, 4, false>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+    else
+      e = launch_pdl(decode_kernel<2, 2, false>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+  }
+
+  __half* xq = reinterpret_cast<__half*>(ws + plan.off_xq);
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return W4A8_ERR_CUDA;
+  CUtensorMap tmap;
+  const cuuint64_t gdim[2] = {cuuint64_t(K), cuuint64_t(M)};
+  const cuuint64_t gstride[1] = {cuuint64_t(K) * 2};
+  const cuuint32_t box[2] = {uint32_t(kTcBK), uint32_t(kTcTokens)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xq, gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return W4A8_ERR_CUDA;
+  TcParams p;
+  p.idx = pk + L.off_idx;
+  p.srel = pk + L.off_srel;
+  p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
+  p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
+  p.s_x = s_x;
+  p.y = y;
+  p.err = d->err;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.C = plan.C;
+  p.T = plan.T;
+  const dim3 grid(unsigned((N + kTcRows - 1) / kTcRows), unsigned((M + kTcTokens - 1) / kTcTokens));
+  const cudaError_t e = launch_pdl(gemm_tc_kernel, grid, dim3(kTcThreads), kTcSmemBytes, s, tmap, p);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* packed, int64_t N, uint16_t* y,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !packed || !y || !workspace) return W4A8_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(y)) return W4A8_ERR_ALIGN;
+  w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
+  if (st != W4A8_OK) return st;
+  return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_get_device_error(void* stream) {
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return W4A8_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return W4A8_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
+  }
+  return (v & kErrTimeout) ? W4A8_ERR_TIMEOUT : W4A8_OK;
+}
+
+const char* w4a8_status_string(w4a8_status status) {
+  switch (status) {
+    case W4A8_OK: return "ok";
+    case W4A8_ERR_NULL: return "a required pointer is NULL";
+    case W4A8_ERR_SHAPE: return "shape outside the supported rules (K % 256, N % 16, K <= 32768, M, N > 0)";
+    case W4A8_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case W4A8_ERR_WORKSPACE: return "buffer smaller than the size function requires";
+    case W4A8_ERR_CUDA: return "a CUDA call failed";
+    case W4A8_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case W4A8_ERR_ARCH: return "the current device is not sm_100";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"
