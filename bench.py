@@ -1,0 +1,421 @@
+"""Benchmark of the asym_w4a8_int8 ConvRot linear layer on B200.
+
+Headline workload: decode GEMV, M=1 token, K=5120, N=17408 (an MLP gate/up
+projection of a 27B hybrid decoder), weights cycled over 8 distinct copies
+(8 x 50.2 MB > the 126 MB L2) so every step streams its weights from HBM.
+A step is one pass of the layer: w4a8_linear (rotate + quantise x, then the
+decode kernel).  Metric: weight GB/s = weight bytes per step / time per step.
+
+Also reported in the same line: the decode kernel timed alone (roofline
+against measured HBM bandwidth), the prefill GEMM at M=4096, K=5120,
+N=17408 (TOPS against the measured dense fp16/bf16 tensor peak), an
+end-to-end figure through the C ABI with host buffers, SM clocks sampled
+during the timed regions, and the CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched by torchrun, one process per GPU; every rank runs an
+independent replica of the workload (the layer needs no exchange between
+GPUs for these shapes), the timed region is bracketed by a barrier and a
+device synchronisation, and the time is the maximum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+M_DEC, K_DEC, N_DEC = 1, 5120, 17408
+M_PRE, K_PRE, N_PRE = 4096, 5120, 17408
+COPIES = 8
+METRIC = "w4a8_linear weight GB/s at M=1 and TOPS at M=4096, % of B200 roofline"
+
+
+def weight_bytes(n: int, k: int) -> int:
+    """Algorithmic bytes of one layer: indices 0.5 B/weight, e4m3 scales
+    1/16 B/weight, fp32 row scales, 16 fp32 levels."""
+    return n * k // 2 + n * k // 16 + 4 * n + 64
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "w4a8_codebook_quantized_rotate_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, files) -> float | None:
+    """DRAM bytes per launch from a committed ncu capture, if the kernel
+    source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_sha256_16") != kernel_source_hash(files):
+        return None
+    return float(d["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self._ok = period_s, threading.Event(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self.nv = None
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self._reasons()
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------- CPU side (oracle)
+
+def oracle_sample(rows: int):
+    """Bounded sample of the decode workload for the CPU oracle: the first
+    ``rows`` output rows of a synthetic C1 layer and one token."""
+    import synth
+    q = synth.quantized_format(N_DEC, K_DEC, synth.rng_for(1, 0, "qfmt"))
+    bits, x, _ = synth.activations(M_DEC, K_DEC, synth.rng_for(1, 0, "act"), K_DEC // 100)
+    return q, x
+
+
+def time_oracle(q, x, rows: int, reps: int):
+    """Oracle linear on ``rows`` output rows, ``reps`` times, one BLAS thread.
+    Returns (seconds per rep, weight bytes per rep)."""
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+    sel = np.arange(rows)
+    with threadpool_limits(limits=1):
+        O.linear_packed(x, q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=sel[: min(rows, 64)])  # warm
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            O.linear_packed(x, q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=sel)
+        dt = (time.perf_counter() - t0) / reps
+    return dt, weight_bytes(rows, K_DEC)
+
+
+def cpu_baseline(budget_s: float = 15.0) -> dict:
+    q, x = oracle_sample(N_DEC)
+    dt1, _ = time_oracle(q, x, 1024, 1)
+    rows = int(min(N_DEC, max(256, 1024 * (budget_s / 3) / max(dt1, 1e-6))))
+    rows -= rows % 16
+    reps = max(1, int(budget_s / max(dt1 * rows / 1024, 1e-6)))
+    reps = min(reps, 5)
+    dt, nbytes = time_oracle(q, x, rows, reps)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle linear (rotate+quantise x, three-tier dequant, fp64 matmul) on {rows} of "
+                      f"{N_DEC} output rows of the M=1 K=5120 layer, {reps} repeats, 1 thread"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    q, x = oracle_sample(N_DEC)
+    # size each step so that warmup + steps take about two minutes in all
+    dt1, _ = time_oracle(q, x, 256, 1)
+    per_row = dt1 / 256
+    rows = int(max(16, min(N_DEC, (120.0 / max(1, args.steps + args.warmup)) / per_row)))
+    rows -= rows % 16
+    rows = max(rows, 16)
+    for _ in range(args.warmup):
+        time_oracle(q, x, rows, 1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(q, x, rows, 1)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = weight_bytes(rows, K_DEC) / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"decode GEMV M={M_DEC} K={K_DEC} N={N_DEC} (bounded row sample per step)",
+                   "rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} of {N_DEC} output rows per step, 1 thread"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- GPU side
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from w4a8_codebook_quantized_rotate_b200 import build as _build
+    from w4a8_codebook_quantized_rotate_b200 import binding as B
+
+    _build.build()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+
+    # ---------------- decode workload: 8 distinct copies of the layer
+    copies = []
+    for c in range(COPIES):
+        q = synth.quantized_format_device(N_DEC, K_DEC, seed=1000 * (rank + 1) + c, device=dev)
+        copies.append(B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"]))
+        del q
+    bits, _, _ = synth.activations(M_DEC, K_DEC, synth.rng_for(1, rank, "act"), K_DEC // 100)
+    x = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    ws = torch.empty(B.linear_workspace_bytes(M_DEC, K_DEC, N_DEC), dtype=torch.uint8, device=dev)
+    y = torch.empty((M_DEC, N_DEC), dtype=torch.bfloat16, device=dev)
+    wbytes = weight_bytes(N_DEC, K_DEC)
+
+    def step(i):
+        B.linear(x, copies[i % COPIES], N_DEC, workspace=ws, out=y)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1))
+        ms_step = ms / args.steps
+        value = world * wbytes * args.steps / (ms * 1e-3) / 1e9
+
+        # decode kernel alone: activations prepared once, then back-to-back runs
+        B.linear_prepare(x, N_DEC, ws)
+        for i in range(args.warmup):
+            B.linear_run(M_DEC, K_DEC, copies[i % COPIES], N_DEC, ws, out=y)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.steps):
+            B.linear_run(M_DEC, K_DEC, copies[i % COPIES], N_DEC, ws, out=y)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gemv_ms = max_over_ranks(g0.elapsed_time(g1)) / args.steps
+    dec_clocks = sampler.summary()
+
+    # ---------------- end to end through the C ABI, host buffers
+    x_host = torch.empty((M_DEC, K_DEC), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(x.cpu())
+    y_host = torch.empty((M_DEC, N_DEC), dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty_like(x)
+    e2e_steps = min(args.steps, 5000)
+
+    def e2e_step(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        B.linear(x_dev, copies[i % COPIES], N_DEC, workspace=ws, out=y)
+        y_host.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    h1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1)) / e2e_steps
+    del copies
+    torch.cuda.empty_cache()
+
+    # ---------------- prefill GEMM, M=4096
+    q = synth.quantized_format_device(N_PRE, K_PRE, seed=77 + rank, device=dev)
+    packed_pre = B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"])
+    del q
+    g = torch.Generator(device=dev)
+    g.manual_seed(5 + rank)
+    xp = torch.randn((M_PRE, K_PRE), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    ws_p = torch.empty(B.linear_workspace_bytes(M_PRE, K_PRE, N_PRE), dtype=torch.uint8, device=dev)
+    yp = torch.empty((M_PRE, N_PRE), dtype=torch.bfloat16, device=dev)
+    flops = 2.0 * M_PRE * N_PRE * K_PRE
+    psampler = ClockSampler(local)
+    with psampler:
+        for _ in range(3):
+            B.linear(xp, packed_pre, N_PRE, workspace=ws_p, out=yp)
+        torch.cuda.synchronize()
+        barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for _ in range(args.prefill_steps):
+            B.linear(xp, packed_pre, N_PRE, workspace=ws_p, out=yp)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        pre_ms = max_over_ranks(p0.elapsed_time(p1)) / args.prefill_steps
+        B.linear_prepare(xp, N_PRE, ws_p)
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for _ in range(args.prefill_steps):
+            B.linear_run(M_PRE, K_PRE, packed_pre, N_PRE, ws_p, out=yp)
+        q1.record(stream)
+        torch.cuda.synchronize()
+        gemm_ms = max_over_ranks(q0.elapsed_time(q1)) / args.prefill_steps
+    pre_clocks = psampler.summary()
+    err = B.get_device_error()
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    achieved = wbytes / (gemv_ms * 1e-3) / 1e9
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16*f16->f32 (4-bit codebook weights, int8 activations, bf16 out)",
+        "data": "synthetic",
+        "config": {
+            "workload": f"decode GEMV M={M_DEC} K={K_DEC} N={N_DEC}, {COPIES} distinct weight copies cycled",
+            "l2": f"inputs larger than L2: {COPIES} x {wbytes / 1e6:.1f} MB weights cycled > 126 MB L2",
+            "weight_bytes_per_step": wbytes,
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+        },
+        "roofline": {
+            "kernel": "decode_kernel (M=1)",
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+            "traffic": profiled_traffic("decode_kernel", ["gemv.cuh", "common.cuh"]),
+            "us_per_launch": gemv_ms * 1e3,
+        },
+        "prefill": {
+            "workload": f"prefill GEMM M={M_PRE} K={K_PRE} N={N_PRE}",
+            "value": flops / (pre_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": pre_ms,
+            "roofline": {"kernel": "gemm_tc_kernel", "bound": "tensor", "achieved": gemm_tflops,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": gemm_tflops / peaks["bf16_tflops"],
+                         "peak_note": "measured dense bf16 burst peak; fp16 kind::f16 runs at the bf16 rate",
+                         "traffic": profiled_traffic("gemm_tc_kernel", ["gemm_tc.cuh", "common.cuh"]),
+                         "ms_per_launch": gemm_ms},
+            "clocks": pre_clocks,
+        },
+        "e2e": {"value": wbytes / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
+                "h2d_bytes_per_step": M_DEC * K_DEC * 2, "d2h_bytes_per_step": M_DEC * N_DEC * 2,
+                "ms_per_step": e2e_ms},
+        "clocks": dec_clocks,
+        "gpu_launches": 2 * args.steps,
+        "device_error": err,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -4,7 +4,9 @@ Bars (the layer's stated tolerances):
   * dequantisation and layout: bit-exact;
   * int8 activations: at most 1 LSB apart, on at most 1e-4 of the elements;
   * linear output (bf16) against the unrounded fp64 oracle: relative L2
-    error <= 2e-3 and, per token m, max |error| <= 1e-2 * ||x_m||_2 * max|W_hat|;
+    error <= 2e-3 and, per token m, max |error| <= 1e-2 * ||x_m||_2 * max|W_hat|
+    (for outputs so small that rounding the exact result to bf16 already
+    costs more than 2e-3, the L2 bar is 1.1x that rounding floor);
   * integer-valued special cases: exact.
 Shapes span several tiles and ragged tails (odd tile counts, token counts
 that are not multiples of 8 or 256) and the full workload shapes (sampled
@@ -44,11 +46,19 @@ def converted(n, k, seed):
     return O.convert_weight(w)
 
 
+def rel_l2_bar(y_ref):
+    """2e-3, unless rounding the exact result itself to bf16 already costs
+    more (outputs of a few dozen elements, where the L2 statistic is noisy):
+    then 1.1x that rounding floor."""
+    floor = np.linalg.norm(O.round_to_bf16(y_ref) - y_ref) / np.linalg.norm(y_ref)
+    return max(REL_L2, 1.1 * floor)
+
+
 def check_linear(y_gpu, y_ref, x, w_maxabs):
     y_gpu = np.asarray(y_gpu, dtype=np.float64)
     err = y_gpu - y_ref
     rel = np.linalg.norm(err) / np.linalg.norm(y_ref)
-    assert rel <= REL_L2, f"relative L2 error {rel:.3e}"
+    assert rel <= rel_l2_bar(y_ref), f"relative L2 error {rel:.3e}"
     bound = MAX_ABS_FACTOR * np.linalg.norm(np.asarray(x, dtype=np.float64), axis=1) * w_maxabs
     worst = np.max(np.abs(err), axis=1)
     assert np.all(worst <= bound), f"max abs error {worst.max():.3e} > bound {bound.min():.3e}"
@@ -218,7 +228,8 @@ def test_linear_deterministic_and_workspace_reuse(lib, layer592, m):
     c, packed, _ = layer592
     bits, _, _ = synth.activations(m, 768, synth.rng_for(8, m, "act"), 8)
     xt = bf16(bits)
-    ws = torch.empty(lib.linear_workspace_bytes(4096, 768, 592) + 4096, dtype=torch.uint8, device="cuda")
+    need = max(lib.linear_workspace_bytes(mm, 768, 592) for mm in (1, 5, 16, 300))
+    ws = torch.empty(need + 4096, dtype=torch.uint8, device="cuda")
     a = lib.linear(xt, packed, 592, workspace=ws).clone()
     # a different shape through the same workspace in between
     other, _, _ = synth.activations(5, 768, synth.rng_for(8, 99, "act"), 8)
