@@ -161,6 +161,37 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
                             void* stream);
 
 /*
+ * w4a8_linear for decode sizes (M <= 16) without any caller-provided
+ * workspace.  The pages have no counterpart to this call; it exists for
+ * callers that cannot allocate device memory where they run the layer: a
+ * plugin whose host application owns the device heap and hands it no
+ * scratch, code on a latency-critical path that must not allocate
+ * (cudaMalloc can synchronise the whole device), or a host program that
+ * drives the library through a foreign-function interface with no device
+ * allocator of its own.
+ *
+ * Instead of a workspace it uses a scratch array built into the library: a
+ * file-scope __device__ array of W4A8_STATIC_SCRATCH_BYTES (16 MiB), which
+ * every GPU that loads the library holds until the process exits.  The call
+ * allocates nothing and calls no allocating routine.  Its first call on a
+ * device looks up the array's device address once (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream
+ * capture.  All calls on a device share the one array and leave their
+ * scratch in it: calls whose work overlaps on the GPU (different streams
+ * without ordering, or other host threads) race and give wrong results, so
+ * order them.  What must start at zero is cleared by each call.
+ *   x, packed, y  as for w4a8_linear (device pointers owned by the caller).
+ * Limits: M <= 16 (larger M returns W4A8_ERR_SHAPE); any shape needing more
+ * scratch than the array holds returns W4A8_ERR_WORKSPACE (no accepted
+ * (N, K) does at M <= 16).
+ * Errors: NULL, SHAPE, WORKSPACE, ALIGN, ARCH, CUDA.
+ */
+#define W4A8_STATIC_SCRATCH_BYTES (16u << 20)
+w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K,
+                                      const void* packed, int64_t N, uint16_t* y,
+                                      void* stream);
+
+/*
  * Synchronise `stream`, then report and clear the device-side error word of
  * the current device: W4A8_ERR_TIMEOUT if a bounded wait inside a kernel
  * gave up since the last call (the affected outputs are then undefined),

@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
+        "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_prepare",
+        "w4a8_linear_run",
         "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
         "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_status_string", "w4a8_unpack_dequant"])
 
@@ -78,6 +79,8 @@ def test_null_and_shape_errors_before_launch(lib):
     assert lib.w4a8_linear_prepare(p, 1, 256, 16, p + 4, 1 << 30, None) == 3
     assert lib.w4a8_linear_run(1, 256, p, 16, p, p, 8, None) == 4
     assert lib.w4a8_linear_run(1, 512, p, 16, None, p, 1 << 30, None) == 1
+    assert lib.w4a8_linear_decode_static(None, 1, 256, p, 16, p, None) == 1
+    assert lib.w4a8_linear_decode_static(p, 17, 256, p, 16, p, None) == 2
 
 
 def test_status_strings(lib):

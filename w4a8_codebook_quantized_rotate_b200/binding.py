@@ -23,7 +23,7 @@ STATUS = {
 EXPORTS = (
     "w4a8_packed_bytes", "w4a8_pack_layout", "w4a8_unpack_dequant", "w4a8_rotate_quant_act",
     "w4a8_linear_workspace_bytes", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
-    "w4a8_get_device_error", "w4a8_status_string",
+    "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_status_string",
 )
 
 _lib = None
@@ -53,6 +53,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_linear": (st, [vp, i64, i64, vp, i64, vp, vp, sz, vp]),
         "w4a8_linear_prepare": (st, [vp, i64, i64, i64, vp, sz, vp]),
         "w4a8_linear_run": (st, [i64, i64, vp, i64, vp, vp, sz, vp]),
+        "w4a8_linear_decode_static": (st, [vp, i64, i64, vp, i64, vp, vp]),
         "w4a8_get_device_error": (st, [vp]),
         "w4a8_status_string": (ctypes.c_char_p, [st]),
     }
@@ -174,6 +175,23 @@ def linear_run(m: int, k: int, packed: torch.Tensor, n: int, workspace: torch.Te
     _cuda(out, torch.bfloat16, "out")
     _check("w4a8_linear_run", lib.w4a8_linear_run(m, k, packed.data_ptr(), n, out.data_ptr(),
                                                   workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out
+
+
+def linear_decode_static(x: torch.Tensor, packed: torch.Tensor, n: int, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """The layer for M <= 16 using the library's built-in device scratch
+    instead of a workspace (for callers that cannot allocate device memory).
+    Calls on one device share that scratch, so they must not overlap on the GPU."""
+    lib = load_library()
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(packed, torch.uint8, "packed")
+    m, k = x.shape
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _cuda(out, torch.bfloat16, "out")
+    _check("w4a8_linear_decode_static", lib.w4a8_linear_decode_static(
+        x.data_ptr(), m, k, packed.data_ptr(), n, out.data_ptr(), _stream(stream)))
     return out
 
 

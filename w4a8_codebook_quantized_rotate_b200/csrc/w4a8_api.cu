@@ -17,6 +17,13 @@ namespace w4a8 {
 // w4a8_get_device_error.
 __device__ unsigned g_error_word;
 
+// Built-in scratch for w4a8_linear_decode_static (callers that cannot
+// allocate device memory).  Every GPU that loads the library holds this
+// array until the process exits.  In host code the name is only a stand-in
+// for the array: its device address comes from cudaGetSymbolAddress.
+constexpr size_t kStaticScratchBytes = size_t(W4A8_STATIC_SCRATCH_BYTES);
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -327,6 +334,34 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* pac
   w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
+}
+
+// Device address of g_static_scratch, looked up once per device with that
+// device current (the first w4a8_linear_decode_static call on the device).
+static void* g_static_scratch_ptr[kMaxDevices];
+static std::mutex g_static_scratch_mutex;
+
+w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, const void* packed, int64_t N,
+                                      uint16_t* y, void* stream) {
+  if (!x || !packed || !y) return W4A8_ERR_NULL;
+  if (M > kDecodeMaxM || !act_shape_ok(M, K) || !weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (linear_plan(M, K, N).total > kStaticScratchBytes) return W4A8_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return W4A8_ERR_CUDA;
+      g_static_scratch_ptr[dev] = p;
+    }
+    scratch = g_static_scratch_ptr[dev];
+  }
+  // The split-K counters the decode kernel needs at zero are cleared by the
+  // activation kernel at the start of every call; nothing else in the
+  // scratch has to start at a known value.
+  return w4a8_linear(x, M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
 }
 
 w4a8_status w4a8_get_device_error(void* stream) {
