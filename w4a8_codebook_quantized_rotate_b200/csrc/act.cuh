@@ -25,7 +25,13 @@ enum ActOut : int {
   kActF16Frag = 2,  // fp16 in mma.sync B-fragment order, the decode kernel's operand
 };
 
-constexpr int kActThreads = 256;
+constexpr int kActMaxThreads = 1024;
+
+// Threads per token: one warp per 256-block, between 256 and 1024.
+__host__ __device__ inline int act_threads(int64_t K) {
+  const int64_t t = 32 * (K / kRotBlock);
+  return int(t < 256 ? 256 : (t > kActMaxThreads ? kActMaxThreads : t));
+}
 
 // Index (in half2 units) of element (m, k) in the decode B-fragment layout:
 // [chunk][n8 block j][lane 32][8 half2], lane = 4 (m % 8) + t, half2
@@ -53,14 +59,17 @@ __device__ __forceinline__ void fwht8_in_lane(float (&v)[8]) {
 }
 
 template <int OUT>
-__global__ void __launch_bounds__(kActThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
+__global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                   void* __restrict__ out, float* __restrict__ s_x,
                                                                   int nb, unsigned* __restrict__ zero_words,
                                                                   int zero_count) {
   extern __shared__ float xr[];  // [K] rotated row
-  __shared__ float warp_max[kActThreads / 32];
-  // Later kernels may start their weight streaming now; they wait for this
-  // grid's completion before reading anything it writes.
+  __shared__ float warp_max[kActMaxThreads / 32];
+  const int nwarps = blockDim.x >> 5;
+  // The previous kernel may still read this workspace: wait for it before
+  // writing.  Then the next kernel may launch (it streams its weights, and
+  // waits for this grid before reading what it writes).
+  pdl_wait();
   pdl_launch_dependents();
   const int m = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -69,7 +78,7 @@ __global__ void __launch_bounds__(kActThreads) rotate_quant_kernel(const uint16_
   }
   const int nblocks = K / kRotBlock;
   float amax = 0.f;
-  for (int b = warp; b < nblocks; b += kActThreads / 32) {
+  for (int b = warp; b < nblocks; b += nwarps) {
     const uint4 raw = *reinterpret_cast<const uint4*>(x + int64_t(m) * K + b * kRotBlock + lane * 8);
     const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
     float v[8];
@@ -103,11 +112,11 @@ __global__ void __launch_bounds__(kActThreads) rotate_quant_kernel(const uint16_
   __syncthreads();
   amax = warp_max[0];
 #pragma unroll
-  for (int i = 1; i < kActThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
+  for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, warp_max[i]);
   const float s = __fdiv_rn(amax, 127.0f);
   if (threadIdx.x == 0) s_x[m] = s;
   // Quantise 8 consecutive values per thread per step.
-  for (int k0 = threadIdx.x * 8; k0 < K; k0 += kActThreads * 8) {
+  for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
     const float4 a = *reinterpret_cast<const float4*>(xr + k0);
     const float4 c = *reinterpret_cast<const float4*>(xr + k0 + 4);
     const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};

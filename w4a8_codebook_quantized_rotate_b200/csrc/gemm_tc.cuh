@@ -32,7 +32,7 @@ constexpr int kTcTokens = 256;    // tokens per tile (MMA N)
 constexpr int kTcBK = 64;         // k per pipeline stage
 constexpr int kTcStagesB = 3;     // x_q stages in shared memory
 constexpr int kTcStagesA = 4;     // expanded-weight stages in TMEM
-constexpr int kTcThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 expansion + epilogue
+constexpr int kTcThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 expansion + epilogue (2 groups)
 constexpr uint32_t kTcStageBBytes = kTcTokens * kTcBK * 2;  // 32 KiB
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcAccCol = 0;     // accumulator: columns [0, 256)
@@ -139,6 +139,7 @@ __device__ __forceinline__ void exp_compute(const ExpStage& e, uint32_t lut_lane
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   extern __shared__ __align__(1024) uint8_t tc_smem[];
+  pdl_launch_dependents();
   TcShared* sh = reinterpret_cast<TcShared*>(tc_smem);
   const uint32_t base = smem_u32(tc_smem);
   // 64 KiB aligned (bits 8..15 zero), past the barrier block
@@ -168,11 +169,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish();
   }
   // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
-  for (int e = threadIdx.x; e < 256 * 32; e += kTcThreads) {
-    const int b = e >> 5;
-    const __half2 h = __floats2half2_rn(p.cb[b & 15], p.cb[b >> 4]);
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(e & 31) * 4u),
-                 "r"(*reinterpret_cast<const uint32_t*>(&h)));
+  // Each lane reads one level once; the pairs come from shuffles.
+  {
+    const float level = p.cb[lane & 15];
+    for (int b = warp; b < 256; b += kTcThreads / 32) {
+      const float lo = __shfl_sync(0xffffffffu, level, b & 15);
+      const float hi = __shfl_sync(0xffffffffu, level, b >> 4);
+      const __half2 h = __floats2half2_rn(lo, hi);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(lane) * 4u),
+                   "r"(*reinterpret_cast<const uint32_t*>(&h)));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -225,6 +231,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------ expansion, then epilogue
+    // Two groups of 4 warps: group G expands the k blocks kb = G, G+2, ...
+    // (each group covers all 128 rows), which doubles the time each warp has
+    // per block; the epilogue splits the 256 accumulator columns between them.
+    const int grp = (warp - 2) >> 2;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = 32 * q + lane;
     const int n = n0 + r;
@@ -235,12 +245,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int PF = 4;
     ExpStage es[PF];
 #pragma unroll
-    for (int i = 0; i < PF; ++i) exp_load(es[i], p, tile, i, g, valid);
+    for (int i = 0; i < PF; ++i) exp_load(es[i], p, tile, grp + 2 * i, g, valid);
     bool ok = true;
-    for (int kb0 = 0; kb0 < KB && ok; kb0 += PF) {
+    for (int kb0 = grp; kb0 < KB && ok; kb0 += 2 * PF) {
 #pragma unroll
       for (int i = 0; i < PF; ++i) {
-        const int kb = kb0 + i;
+        const int kb = kb0 + 2 * i;
         if (kb < KB && ok) {
           const int sa = kb % kTcStagesA;
           uint32_t v[32];
@@ -249,7 +259,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) v[c] = 0u;
           }
-          exp_load(es[i], p, tile, kb + PF, g, valid);
+          exp_load(es[i], p, tile, kb + 2 * PF, g, valid);
           // lane 0 polls; the verdict is made warp-uniform before the
           // .sync.aligned TMEM store
           int w_ok = lane == 0 ? int(tc_wait(&sh->a_empty[sa], ((kb / kTcStagesA) & 1) ^ 1, sh, p.err)) : 0;
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       pdl_wait();  // s_x comes from the previous kernel
       const float sch = valid ? p.sch[n] : 0.f;
 #pragma unroll 1
-      for (int ci = 0; ci < kTcTokens / 32; ++ci) {
+      for (int ci = grp * (kTcTokens / 64); ci < (grp + 1) * (kTcTokens / 64); ++ci) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + trow + kTcAccCol + uint32_t(ci) * 32u, v);
         tc_wait_ld();

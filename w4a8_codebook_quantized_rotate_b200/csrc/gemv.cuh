@@ -19,11 +19,14 @@
 //
 // Work split ("stream-K"): a unit is (tile pair p, chunk c), i.e. 32 rows x
 // 64 k.  The P * C units, in [p][c] order (the order they lie in memory),
-// are cut into W equal ranges, one per warp.  A warp that covers a whole
-// tile pair writes y directly; a pair split across warps leaves one fp32
-// partial per warp in the workspace, and the last of its warps to finish
-// (found with an atomic counter, no waiting) adds the partials in warp order
-// -- the sum is deterministic -- and writes y.
+// are cut into W equal ranges, one per warp; a CTA's 16 warps hold 16
+// consecutive ranges.  A warp that covers a whole tile pair writes y
+// directly.  A pair split between warps is reduced in two levels, both in a
+// fixed order (the result is deterministic): the warps of a CTA leave their
+// partials in shared memory and one warp adds them after a CTA barrier; a
+// pair that also crosses into another CTA leaves one partial per CTA in the
+// workspace, and the last CTA to finish it (an atomic counter, no waiting)
+// adds those and writes y.
 #pragma once
 
 #include "common.cuh"
@@ -32,9 +35,10 @@ namespace w4a8 {
 
 constexpr int kDecWarps = 16;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecTG = 2;                    // tiles (16 rows each) per unit
-constexpr int kDecMaxWarps = 148 * kDecWarps;  // cap on W, fixes the workspace size
-constexpr size_t kDecSmemBytes = 2 * 65536;  // room for a 64 KiB-aligned 64 KiB table
+constexpr int kDecTG = 2;                          // tiles (16 rows each) per unit
+constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
+constexpr int kDecMaxWarps = kDecMaxCtas * kDecWarps;
+constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
 
 struct DecodeParams {
   const uint8_t* idx;    // index plane
@@ -44,19 +48,24 @@ struct DecodeParams {
   const uint4* xfrag;    // activations in B-fragment order, [C][NB][32][2] uint4
   const float* s_x;      // [M]
   uint16_t* y;           // [M, N] bf16
-  float* slots;          // [2 W][kDecTG * 16 * 8 * NB]
+  float* slots;          // [2 * CTAs][kDecTG * 16][M]: per-CTA partials of pairs shared with other CTAs
   unsigned* counters;    // [P]
   unsigned* err;
   int M, N, C, T, P, W, U;
 };
 
-__host__ __device__ inline int dec_slot_floats(int nb) { return kDecTG * 16 * 8 * nb; }
+// Floats of one partial (a tile pair, the first M tokens).
+__host__ __device__ inline int dec_slot_floats(int m) { return kDecTG * 16 * m; }
 
-// The warp whose range holds unit u (ranges are [floor(w U / W), floor((w+1) U / W))).
-__device__ __forceinline__ int dec_warp_of(int u, int U, int W) {
-  return int((int64_t(u + 1) * W - 1) / U);
+// Dynamic shared memory of a launch: table (+ alignment room), one token's
+// activations, and the CTA's per-warp partials.
+__host__ __device__ inline size_t dec_smem_bytes(int m, int k, bool single) {
+  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(kDecWarps) * 2 * dec_slot_floats(m) * 4;
 }
+
+// Ranges: warp w holds units [floor(w U / W), floor((w+1) U / W)).
 __device__ __forceinline__ int dec_range_begin(int w, int U, int W) { return int(int64_t(w) * U / W); }
+__device__ __forceinline__ int dec_warp_of(int u, int U, int W) { return int((int64_t(u + 1) * W - 1) / U); }
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;
@@ -75,93 +84,160 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128_(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// D = A B + 0, with the zero C operand passed in as a register the caller
+// keeps for the whole loop.
+__device__ __forceinline__ void mma_16816z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1, float z) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%10, %10, %10, %10};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-template <int NB>
+// Per-unit registers: index bytes and group scales of the two tiles, and (for
+// more than one token) the B fragments of the unit's chunk.
+template <int NB, bool SINGLE>
 struct DecStage {
-  uint4 w[kDecTG];     // index bytes, one 16-byte fragment set per tile
-  uint2 s[kDecTG];     // group-scale bytes (rows g, g+8) x 4 steps
-  uint4 x[NB][2];      // B fragments for the chunk's four k16 steps
+  uint4 w[kDecTG];
+  uint2 s[kDecTG];
+  uint4 x[SINGLE ? 1 : NB][2];
 };
 
-template <int NB>
-__device__ __forceinline__ void dec_load_weights(DecStage<NB>& st, const DecodeParams& p, int pair, int c,
-                                                 int lane) {
-#pragma unroll
-  for (int i = 0; i < kDecTG; ++i) {
-    const int tile = pair * kDecTG + i;
-    if (tile < p.T) {
-      const size_t blk = size_t(tile) * p.C + c;
-      st.w[i] = ld_stream_v4(p.idx + blk * kChunkIdxBytes + lane * 16);
-      st.s[i] = ld_stream_v2(p.srel + blk * kChunkSrelBytes + (lane >> 2) * 8);
-    } else {
-      st.w[i] = make_uint4(0, 0, 0, 0);
-      st.s[i] = make_uint2(0, 0);
-    }
-  }
+// Where the next unit to prefetch lies.  The second tile of a pair sits
+// C blocks after the first; for an odd tile count the missing last tile
+// re-reads the first (its results are never stored).
+struct DecCursor {
+  const uint8_t* idx;   // this lane's 16 bytes of tile 0
+  const uint8_t* srel;  // this lane's 8 scale bytes of tile 0
+  uint32_t idx1, srel1; // byte offsets of tile 1
+  int pair, c;
+};
+
+__device__ __forceinline__ void dec_cursor_pair(DecCursor& q, const DecodeParams& p) {
+  const bool two = q.pair * kDecTG + 1 < p.T;
+  q.idx1 = two ? uint32_t(p.C) * kChunkIdxBytes : 0u;
+  q.srel1 = two ? uint32_t(p.C) * kChunkSrelBytes : 0u;
 }
 
-template <int NB>
-__device__ __forceinline__ void dec_load_x(DecStage<NB>& st, const DecodeParams& p, int c, int lane) {
-#pragma unroll
-  for (int j = 0; j < NB; ++j) {
-    if ((lane >> 2) + 8 * j < p.M) {
-      const uint4* src = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
-      st.x[j][0] = __ldg(src);
-      st.x[j][1] = __ldg(src + 1);
-    } else {
-      st.x[j][0] = make_uint4(0, 0, 0, 0);
-      st.x[j][1] = make_uint4(0, 0, 0, 0);
-    }
+__device__ __forceinline__ void dec_cursor_advance(DecCursor& q, const DecodeParams& p) {
+  q.idx += kChunkIdxBytes;
+  q.srel += kChunkSrelBytes;
+  if (++q.c == p.C) {
+    q.c = 0;
+    ++q.pair;
+    q.idx += size_t(p.C) * kChunkIdxBytes;  // skip the previous pair's second tile
+    q.srel += size_t(p.C) * kChunkSrelBytes;
+    dec_cursor_pair(q, p);
   }
 }
 
 template <int NB, bool SINGLE>
-__device__ __forceinline__ void dec_compute(const DecStage<NB>& st, float (&acc)[kDecTG][NB][4],
-                                            uint32_t lut_lane) {
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    uint32_t b[NB][2];
+__device__ __forceinline__ void dec_load(DecStage<NB, SINGLE>& st, const DecCursor& q, const DecodeParams& p,
+                                         int lane) {
+  st.w[0] = ld_stream_v4(q.idx);
+  st.w[1] = ld_stream_v4(q.idx + q.idx1);
+  st.s[0] = ld_stream_v2(q.srel);
+  st.s[1] = ld_stream_v2(q.srel + q.srel1);
+  if constexpr (!SINGLE) {
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-      const uint4& xv = st.x[j][s >> 1];
-      b[j][0] = (s & 1) ? xv.z : xv.x;
-      b[j][1] = (s & 1) ? xv.w : xv.y;
+      if ((lane >> 2) + 8 * j < p.M) {
+        const uint4* src = p.xfrag + (size_t(q.c * NB + j) * 32 + lane) * 2;
+        st.x[j][0] = __ldg(src);
+        st.x[j][1] = __ldg(src + 1);
+      } else {
+        st.x[j][0] = make_uint4(0, 0, 0, 0);
+        st.x[j][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+}
+
+// One unit: all 32 table lookups (and, for one token, the 4 B fragments from
+// shared memory) are issued first, back to back, so their latencies overlap;
+// then the 8 (x NB) MMAs and the fp32 group-scale accumulation.
+template <int NB, bool SINGLE>
+__device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, float (&acc)[kDecTG][NB][4],
+                                            uint32_t lut_lane, uint32_t xs_chunk) {
+  const float zero = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {  // two halves of two k16 steps each
+    uint32_t a[kDecTG][2][4];
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int s = 2 * h + s2;
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i) {
+        const uint32_t word = s == 0 ? st.w[i].x : s == 1 ? st.w[i].y : s == 2 ? st.w[i].z : st.w[i].w;
+        // address = table base + (byte << 8) + 4 lane: the byte replaces bits 8..15
+        a[i][s2][0] = lds32(prmt(word, lut_lane, 0x7604u));
+        a[i][s2][1] = lds32(prmt(word, lut_lane, 0x7614u));
+        a[i][s2][2] = lds32(prmt(word, lut_lane, 0x7624u));
+        a[i][s2][3] = lds32(prmt(word, lut_lane, 0x7634u));
+      }
+    }
+    uint32_t b[2][NB][2];
+    if constexpr (SINGLE) {
+      const uint4 v = lds128_(xs_chunk + 16u * h);
+      b[0][0][0] = v.x;
+      b[0][0][1] = v.y;
+      b[1][0][0] = v.z;
+      b[1][0][1] = v.w;
+    } else {
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          const uint4& xv = st.x[j][h];
+          b[s2][j][0] = s2 ? xv.z : xv.x;
+          b[s2][j][1] = s2 ? xv.w : xv.y;
+        }
     }
 #pragma unroll
-    for (int i = 0; i < kDecTG; ++i) {
-      const uint32_t word = s == 0 ? st.w[i].x : s == 1 ? st.w[i].y : s == 2 ? st.w[i].z : st.w[i].w;
-      // address = lut base + (byte << 8) + 4 lane: the byte replaces bits 8..15
-      const uint32_t a0 = lds32(prmt(word, lut_lane, 0x7604u));
-      const uint32_t a1 = lds32(prmt(word, lut_lane, 0x7614u));
-      const uint32_t a2 = lds32(prmt(word, lut_lane, 0x7624u));
-      const uint32_t a3 = lds32(prmt(word, lut_lane, 0x7634u));
-      const uint32_t pair_codes = ((s < 2) ? st.s[i].x : st.s[i].y) >> (16 * (s & 1));
-      const float2 sc = e4m3x2_to_float2(pair_codes);  // (row g, row g+8)
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int s = 2 * h + s2;
 #pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        float d[4];
-        mma_16816(d, a0, a1, a2, a3, b[j][0], b[j][1]);
-        acc[i][j][0] = fmaf(d[0], sc.x, acc[i][j][0]);
-        acc[i][j][2] = fmaf(d[2], sc.y, acc[i][j][2]);
-        if (!SINGLE) {
-          acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
-          acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
+      for (int i = 0; i < kDecTG; ++i) {
+        const uint32_t pair_codes = ((s < 2) ? st.s[i].x : st.s[i].y) >> (16 * (s & 1));
+        const float2 sc = e4m3x2_to_float2(pair_codes);  // (row g, row g+8)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          float d[4];
+          mma_16816z(d, a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b[s2][j][0], b[s2][j][1], zero);
+          acc[i][j][0] = fmaf(d[0], sc.x, acc[i][j][0]);
+          acc[i][j][2] = fmaf(d[2], sc.y, acc[i][j][2]);
+          if (!SINGLE) {
+            acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
+            acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
+          }
         }
       }
     }
   }
 }
 
-// acc element e of (tile i, block j) is row 16 tile + g + 8 (e >> 1), token 8 j + 2 t + (e & 1).
+// acc element e of (tile i, block j) is row 16 (2 pair + i) + g + 8 (e >> 1),
+// token 8 j + 2 t + (e & 1).
 template <int NB>
 __device__ __forceinline__ void dec_epilogue(const float (&acc)[kDecTG][NB][4], const DecodeParams& p, int pair,
                                              int lane) {
@@ -185,24 +261,12 @@ __device__ __forceinline__ void dec_epilogue(const float (&acc)[kDecTG][NB][4], 
   }
 }
 
+// A partial lives as [tile i][row 16][token m] floats; each lane owns the
+// entries of its fragment positions with token < M.
 template <int NB>
-__device__ __forceinline__ int dec_slot_index(int w, int pair, const DecodeParams& p) {
-  const int first_pair = dec_range_begin(w, p.U, p.W) / p.C;
-  return 2 * w + (pair == first_pair ? 0 : 1);
-}
-
-// Called when a warp leaves tile pair `pair`, having covered chunks
-// [c_first, c_last] of it.
-template <int NB>
-__device__ __forceinline__ void dec_flush(float (&acc)[kDecTG][NB][4], const DecodeParams& p, int pair,
-                                          int c_first, int c_last, int w, int lane) {
-  if (c_first == 0 && c_last == p.C - 1) {
-    dec_epilogue<NB>(acc, p, pair, lane);
-    return;
-  }
+__device__ __forceinline__ void dec_partial_store_smem(const float (&acc)[kDecTG][NB][4], uint32_t dst, int M,
+                                                       int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int sf = dec_slot_floats(NB);
-  float* mine = p.slots + size_t(dec_slot_index<NB>(w, pair, p)) * sf;
 #pragma unroll
   for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
@@ -210,26 +274,211 @@ __device__ __forceinline__ void dec_flush(float (&acc)[kDecTG][NB][4], const Dec
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = 8 * j + 2 * t + (e & 1);
-        if (tok < p.M) mine[(i * 16 + g + 8 * (e >> 1)) * (8 * NB) + tok] = acc[i][j][e];
+        if (tok < M) {
+          const uint32_t a = dst + uint32_t(((i * 16 + g + 8 * (e >> 1)) * M + tok) * 4);
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(acc[i][j][e]));
+        }
       }
-  __threadfence();
-  __syncwarp();
-  const int w_first = dec_warp_of(pair * p.C, p.U, p.W);
-  const int w_last = dec_warp_of(pair * p.C + p.C - 1, p.U, p.W);
-  unsigned old = 0;
-  if (lane == 0) old = atomicAdd(p.counters + pair, 1u);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (old != unsigned(w_last - w_first)) return;
-  __threadfence();
-  float sum[kDecTG][NB][4];
+}
+
+template <int NB>
+__device__ __forceinline__ void dec_partial_add_smem(float (&acc)[kDecTG][NB][4], uint32_t src, int M, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
     for (int j = 0; j < NB; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sum[i][j][e] = 0.f;
-  for (int ww = w_first; ww <= w_last; ++ww) {
-    const float* src = p.slots + size_t(dec_slot_index<NB>(ww, pair, p)) * sf;
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 8 * j + 2 * t + (e & 1);
+        if (tok < M) {
+          float v;
+          asm volatile("ld.shared.f32 %0, [%1];"
+                       : "=f"(v)
+                       : "r"(src + uint32_t(((i * 16 + g + 8 * (e >> 1)) * M + tok) * 4)));
+          acc[i][j][e] += v;
+        }
+      }
+}
+
+template <int NB>
+__device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
+#pragma unroll
+  for (int i = 0; i < kDecTG; ++i)
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+}
+
+template <int NB, int D, bool SINGLE>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t dec_smem[];
+  // The next kernel may launch now: it streams its own weights and waits for
+  // this grid's completion before it touches anything this grid writes.
+  pdl_launch_dependents();
+  const uint32_t base = smem_u32(dec_smem);
+  const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned: bits 8..15 are zero
+  const uint32_t xs = lut + 65536u;                   // one token: x staged here (2 K bytes)
+  const uint32_t parts = xs + (SINGLE ? uint32_t(p.C) * 128u : 0u);  // [warp][2] partials
+  const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int w = blockIdx.x * kDecWarps + wl;
+  const bool active = w < p.W;
+  const int u0 = active ? dec_range_begin(w, p.U, p.W) : 0;
+  const int u1 = active ? dec_range_begin(w + 1, p.U, p.W) : 0;
+  const int n_units = u1 - u0;
+
+  DecCursor q;
+  q.pair = u0 / p.C;
+  q.c = u0 - q.pair * p.C;
+  {
+    const size_t blk = size_t(q.pair) * kDecTG * p.C + q.c;
+    q.idx = p.idx + blk * kChunkIdxBytes + lane * 16;
+    q.srel = p.srel + blk * kChunkSrelBytes + (lane >> 2) * 8;
+  }
+  dec_cursor_pair(q, p);
+  const int first_pair = q.pair;
+  const int first_c = q.c;
+
+  DecStage<NB, SINGLE> st[D];
+  // Weights do not depend on the previous kernel: start streaming them first.
+  // (x for more than one token comes from it, so it is loaded after the wait.)
+#pragma unroll
+  for (int d = 0; d < D; ++d) {
+    if (d < n_units) {
+      st[d].w[0] = ld_stream_v4(q.idx);
+      st[d].w[1] = ld_stream_v4(q.idx + q.idx1);
+      st[d].s[0] = ld_stream_v2(q.srel);
+      st[d].s[1] = ld_stream_v2(q.srel + q.srel1);
+      dec_cursor_advance(q, p);
+    }
+  }
+  // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
+  {
+    const float level = p.cb[lane & 15];
+    for (int b = wl; b < 256; b += kDecWarps) {
+      const float lo = __shfl_sync(0xffffffffu, level, b & 15);
+      const float hi = __shfl_sync(0xffffffffu, level, b >> 4);
+      const __half2 h = __floats2half2_rn(lo, hi);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(lane) * 4u),
+                   "r"(*reinterpret_cast<const uint32_t*>(&h)));
+    }
+  }
+  pdl_wait();  // activations, scales and counters come from the previous kernel
+  if constexpr (SINGLE) {
+    // token 0's B fragments: per chunk, lanes t = 0..3 of the fragment layout (128 bytes)
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.xfrag);
+    for (int e = threadIdx.x; e < p.C * 8; e += kDecThreads) {
+      const int c = e >> 3, qq = e & 7;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + size_t(c) * 1024 + qq * 16));
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + uint32_t(c) * 128u + uint32_t(qq) * 16u),
+                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+    }
+  } else {
+    int c = first_c;
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      if (d < n_units) {
+        if constexpr (!SINGLE) {
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            if ((lane >> 2) + 8 * j < p.M) {
+              const uint4* srcx = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
+              st[d].x[j][0] = __ldg(srcx);
+              st[d].x[j][1] = __ldg(srcx + 1);
+            } else {
+              st[d].x[j][0] = make_uint4(0, 0, 0, 0);
+              st[d].x[j][1] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        if (++c == p.C) c = 0;
+      }
+    }
+  }
+  __syncthreads();
+
+  const uint32_t lut_lane = lut + uint32_t(lane) * 4u;
+  const uint32_t xs_lane = xs + uint32_t(lane & 3) * 32u;
+  float acc[kDecTG][NB][4];
+  dec_zero<NB>(acc);
+  int cur_pair = first_pair, cur_c = first_c, c_first = first_c;
+  // A finished or range-ending pair: write y if this warp covered all of it,
+  // else park the partial in shared memory (slot 0: the warp's first pair).
+  auto close_pair = [&](int c_last) {
+    if (c_first == 0 && c_last == p.C - 1) {
+      dec_epilogue<NB>(acc, p, cur_pair, lane);
+    } else {
+      const uint32_t slot = parts + uint32_t(wl * 2 + (cur_pair == first_pair ? 0 : 1)) * part_bytes;
+      dec_partial_store_smem<NB>(acc, slot, p.M, lane);
+    }
+  };
+
+  auto unit_done = [&]() {
+    if (++cur_c == p.C) {
+      close_pair(p.C - 1);
+      dec_zero<NB>(acc);
+      cur_c = 0;
+      ++cur_pair;
+      c_first = 0;
+    }
+  };
+  int ub = 0;
+  // Full rounds: every stage computes and refills.
+  for (; ub + 2 * D <= n_units; ub += D) {
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
+      dec_load<NB, SINGLE>(st[d], q, p, lane);
+      dec_cursor_advance(q, p);
+      unit_done();
+    }
+  }
+  // Tail: fewer than 2 D units left.
+#pragma unroll
+  for (int d2 = 0; d2 < 2 * D; ++d2) {
+    const int d = d2 % D;
+    if (ub + d2 < n_units) {
+      dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
+      if (ub + d2 + D < n_units) {
+        dec_load<NB, SINGLE>(st[d], q, p, lane);
+        dec_cursor_advance(q, p);
+      }
+      unit_done();
+    }
+  }
+  if (n_units > 0 && cur_c != 0) close_pair(cur_c - 1);
+  __syncthreads();
+
+  // ---- level 2: pairs split between warps, reduced by one warp of the CTA
+  const int cta_w0 = blockIdx.x * kDecWarps;
+  const int cta_w1 = min(cta_w0 + kDecWarps, p.W);  // exclusive
+  if (cta_w0 >= cta_w1) return;
+  const int v0 = dec_range_begin(cta_w0, p.U, p.W);
+  const int v1 = dec_range_begin(cta_w1, p.U, p.W);
+  const int pair_lo = v0 / p.C, pair_hi = (v1 - 1) / p.C;
+  for (int pr = pair_lo + wl; pr <= pair_hi; pr += kDecWarps) {
+    const int wf = dec_warp_of(pr * p.C, p.U, p.W);            // first warp holding this pair
+    const int wlst = dec_warp_of(pr * p.C + p.C - 1, p.U, p.W);  // last warp holding it
+    if (wf == wlst) continue;                                    // one warp held all of it: done
+    const int a = max(wf, cta_w0), z = min(wlst, cta_w1 - 1);     // this CTA's contributors
+    dec_zero<NB>(acc);
+    for (int ww = a; ww <= z; ++ww) {
+      const int first_of_ww = dec_range_begin(ww, p.U, p.W) / p.C;
+      const uint32_t slot = parts + uint32_t((ww - cta_w0) * 2 + (pr == first_of_ww ? 0 : 1)) * part_bytes;
+      dec_partial_add_smem<NB>(acc, slot, p.M, lane);
+    }
+    const int cf = dec_warp_of(pr * p.C, p.U, p.W) / kDecWarps;             // first CTA holding the pair
+    const int cl = dec_warp_of(pr * p.C + p.C - 1, p.U, p.W) / kDecWarps;   // last CTA holding it
+    if (cf == cl) {
+      dec_epilogue<NB>(acc, p, pr, lane);
+      continue;
+    }
+    // ---- level 3: the pair spans CTAs; park this CTA's partial in the workspace
+    const int sf = dec_slot_floats(p.M);
+    const int g = lane >> 2, t = lane & 3;
+    float* mine = p.slots + size_t(blockIdx.x * 2 + (pr == pair_lo ? 0 : 1)) * sf;
 #pragma unroll
     for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
@@ -237,96 +486,48 @@ __device__ __forceinline__ void dec_flush(float (&acc)[kDecTG][NB][4], const Dec
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int tok = 8 * j + 2 * t + (e & 1);
-          if (tok < p.M) sum[i][j][e] += __ldcg(src + (i * 16 + g + 8 * (e >> 1)) * (8 * NB) + tok);
+          if (tok < p.M) mine[(i * 16 + g + 8 * (e >> 1)) * p.M + tok] = acc[i][j][e];
         }
-  }
-  if (lane == 0) p.counters[pair] = 0u;  // ready for the next launch on this workspace
-  dec_epilogue<NB>(sum, p, pair, lane);
-}
-
-template <int NB, int D, bool SINGLE>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
-  extern __shared__ __align__(16) uint8_t dec_smem[];
-  const uint32_t base = smem_u32(dec_smem);
-  const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned: bits 8..15 are zero
-  const int lane = threadIdx.x & 31;
-  // Fill the table: entry b, lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
-  for (int e = threadIdx.x; e < 256 * 32; e += kDecThreads) {
-    const int b = e >> 5;
-    const __half2 h = __floats2half2_rn(p.cb[b & 15], p.cb[b >> 4]);
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(e & 31) * 4u),
-                 "r"(*reinterpret_cast<const uint32_t*>(&h)));
-  }
-  __syncthreads();
-  const uint32_t lut_lane = lut + uint32_t(lane) * 4u;
-  const int w = blockIdx.x * kDecWarps + (threadIdx.x >> 5);
-  if (w >= p.W) return;
-  const int u0 = dec_range_begin(w, p.U, p.W);
-  const int u1 = dec_range_begin(w + 1, p.U, p.W);
-
-  DecStage<NB> st[D];
-  // Weights do not depend on the previous kernel: start streaming them now.
-  {
-    int pr = u0 / p.C, c = u0 - pr * p.C;
+    __threadfence();
+    __syncwarp();
+    unsigned old = 0;
+    if (lane == 0) old = atomicAdd(p.counters + pr, 1u);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != unsigned(cl - cf)) continue;  // another CTA finishes this pair
+    __threadfence();
+    // Sum the CTAs' partials in CTA order; all loads are independent.
+    constexpr int kMaxCtaParts = 8 / NB;
+    dec_zero<NB>(acc);
+    for (int c0 = cf; c0 <= cl; c0 += kMaxCtaParts) {
+      float v[kMaxCtaParts][kDecTG][NB][4];
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      if (u0 + d < u1) dec_load_weights<NB>(st[d], p, pr, c, lane);
-      if (++c == p.C) { c = 0; ++pr; }
-    }
-  }
-  pdl_wait();  // activations, scales and counters come from the previous kernel
-  {
-    int c = u0 % p.C;
+      for (int r = 0; r < kMaxCtaParts; ++r) {
+        const int cc = c0 + r;
+        const bool have = cc <= cl;
+        const int first_of_cc = dec_range_begin(cc * kDecWarps, p.U, p.W) / p.C;
+        const float* src = p.slots + size_t(cc * 2 + (pr == first_of_cc ? 0 : 1)) * sf;
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      if (u0 + d < u1) dec_load_x<NB>(st[d], p, c, lane);
-      if (++c == p.C) c = 0;
-    }
-  }
-
-  float acc[kDecTG][NB][4];
+        for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
-  for (int i = 0; i < kDecTG; ++i)
+          for (int j = 0; j < NB; ++j)
 #pragma unroll
-    for (int j = 0; j < NB; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-  int cur_pair = u0 / p.C;
-  int cur_c = u0 - cur_pair * p.C;  // chunk of the unit being computed
-  int c_first = cur_c;
-  // position of the unit being prefetched (u + D)
-  int pf_pair = (u0 + D) / p.C;
-  int pf_c = (u0 + D) - pf_pair * p.C;
-
-  for (int ub = u0; ub < u1; ub += D) {
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int u = ub + d;
-      if (u < u1) {
-        if (cur_c == 0 && u != u0) {  // entered a new tile pair
-          dec_flush<NB>(acc, p, cur_pair - 1, c_first, p.C - 1, w, lane);
-#pragma unroll
-          for (int i = 0; i < kDecTG; ++i)
-#pragma unroll
-            for (int j = 0; j < NB; ++j)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-          c_first = 0;
-        }
-        dec_compute<NB, SINGLE>(st[d], acc, lut_lane);
-        if (u + D < u1) {
-          dec_load_weights<NB>(st[d], p, pf_pair, pf_c, lane);
-          dec_load_x<NB>(st[d], p, pf_c, lane);
-        }
-        if (++pf_c == p.C) { pf_c = 0; ++pf_pair; }
-        if (++cur_c == p.C) { cur_c = 0; ++cur_pair; }
+            for (int e = 0; e < 4; ++e) {
+              const int tok = 8 * j + 2 * t + (e & 1);
+              v[r][i][j][e] = (have && tok < p.M) ? __ldcg(src + (i * 16 + g + 8 * (e >> 1)) * p.M + tok) : 0.f;
+            }
       }
+#pragma unroll
+      for (int r = 0; r < kMaxCtaParts; ++r)
+#pragma unroll
+        for (int i = 0; i < kDecTG; ++i)
+#pragma unroll
+          for (int j = 0; j < NB; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] += v[r][i][j][e];
     }
+    if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
+    dec_epilogue<NB>(acc, p, pr, lane);
   }
-  // The last unit computed was u1 - 1; its pair is the one still open.
-  const int last_pair = (u1 - 1) / p.C;
-  dec_flush<NB>(acc, p, last_pair, c_first, (u1 - 1) - last_pair * p.C, w, lane);
 }
 
 }  // namespace w4a8

@@ -75,9 +75,9 @@ w4a8_status device_state(DeviceState** out) {
       if (allow_smem(rotate_quant_kernel<kActI8Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Frag>, size_t(kMaxK) * 4) != cudaSuccess ||
-          allow_smem(decode_kernel<1, 4, true>, kDecSmemBytes) != cudaSuccess ||
-          allow_smem(decode_kernel<1, 4, false>, kDecSmemBytes) != cudaSuccess ||
-          allow_smem(decode_kernel<2, 2, false>, kDecSmemBytes) != cudaSuccess ||
+          allow_smem(decode_kernel<1, 4, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
+          allow_smem(decode_kernel<1, 3, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<2, 2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
         return W4A8_ERR_CUDA;
     }
@@ -113,7 +113,7 @@ LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
     L.off_xq = 256;
     L.off_cnt = round_up(L.off_xq + size_t(K) * L.nb * 16, 256);
     L.off_slots = round_up(L.off_cnt + size_t(L.P) * 4, 256);
-    L.total = round_up(L.off_slots + size_t(2) * kDecMaxWarps * dec_slot_floats(L.nb) * 4, 256);
+    L.total = round_up(L.off_slots + size_t(2) * kDecMaxCtas * dec_slot_floats(int(M)) * 4, 256);
   } else {
     L.nb = 0;
     L.off_sx = 0;
@@ -213,7 +213,7 @@ w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_
   if (!aligned16(x) || !aligned16(x_q) || !aligned16(s_x)) return W4A8_ERR_ALIGN;
   DeviceState* d = nullptr;
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
-  rotate_quant_kernel<kActI8Row><<<unsigned(M), kActThreads, size_t(K) * 4, static_cast<cudaStream_t>(stream)>>>(
+  rotate_quant_kernel<kActI8Row><<<unsigned(M), act_threads(K), size_t(K) * 4, static_cast<cudaStream_t>(stream)>>>(
       x, int(M), int(K), x_q, s_x, 0, nullptr, 0);
   return launch_status();
 }
@@ -244,11 +244,14 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* s_x = reinterpret_cast<float*>(ws + plan.off_sx);
   if (plan.decode) {
-    rotate_quant_kernel<kActF16Frag><<<unsigned(M), kActThreads, size_t(K) * 4, s>>>(
-        x, int(M), int(K), ws + plan.off_xq, s_x, plan.nb, reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P);
+    if (launch_pdl(rotate_quant_kernel<kActF16Frag>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
+                   int(M), int(K), (void*)(ws + plan.off_xq), s_x, plan.nb,
+                   reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P) != cudaSuccess)
+      return W4A8_ERR_CUDA;
   } else {
-    rotate_quant_kernel<kActF16Row><<<unsigned(M), kActThreads, size_t(K) * 4, s>>>(
-        x, int(M), int(K), ws + plan.off_xq, s_x, 0, nullptr, 0);
+    if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
+                   int(M), int(K), (void*)(ws + plan.off_xq), s_x, 0, (unsigned*)nullptr, 0) != cudaSuccess)
+      return W4A8_ERR_CUDA;
   }
   return launch_status();
 }
@@ -284,16 +287,17 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
     p.T = plan.T;
     p.P = plan.P;
     p.U = plan.P * plan.C;
-    const int warps_avail = (d->sms < 148 ? d->sms : 148) * kDecWarps;
+    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
     p.W = p.U < warps_avail ? p.U : warps_avail;
     const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
     cudaError_t e;
+    const size_t smem = dec_smem_bytes(int(M), int(K), M == 1);
     if (plan.nb == 1 && M == 1)
-      e = launch_pdl(decode_kernel<1, 4, true>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+      e = launch_pdl(decode_kernel<1, 4, true>, grid, dim3(kDecThreads), smem, s, p);
     else if (plan.nb == 1)
-      e = launch_pdl(decode_kernel<1, 4, false>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+      e = launch_pdl(decode_kernel<1, 3, false>, grid, dim3(kDecThreads), smem, s, p);
     else
-      e = launch_pdl(decode_kernel<2, 2, false>, grid, dim3(kDecThreads), kDecSmemBytes, s, p);
+      e = launch_pdl(decode_kernel<2, 2, false>, grid, dim3(kDecThreads), smem, s, p);
     return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
   }
 
