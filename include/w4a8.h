@@ -62,7 +62,9 @@ typedef enum w4a8_status {
  * Size in bytes of the device layout produced by w4a8_pack_layout for an
  * [N, K] weight, or 0 if (N, K) break the shape rules.  About 0.5625 bytes
  * per weight (0.5 for the indices, 1/16 for the group scales) plus 4 bytes
- * per row and 64 bytes for the codebook, each region padded to 256 bytes.
+ * per row and 64 bytes for the codebook, each region padded to 256 bytes;
+ * rows are stored in blocks of 32, so an N that is an odd multiple of 16
+ * carries 16 rows of zero padding.
  */
 size_t w4a8_packed_bytes(int64_t N, int64_t K);
 
@@ -117,8 +119,13 @@ w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K,
 /*
  * Bytes of device workspace w4a8_linear needs for (M, K, N), or 0 if the
  * shape breaks the rules.  The workspace holds the quantised activations,
- * their scales and the split-K partial sums; its content need not be
- * initialised and is scratch between calls.
+ * their scales, the split-K partial sums and the split-K arrival counters.
+ * Fill a new workspace with zeros before its first use (for example
+ * cudaMemsetAsync): the one-token path of w4a8_linear needs the counters at
+ * zero when it starts, and every completed call leaves them at zero again
+ * (w4a8_linear_prepare also clears them).  After a call that reported
+ * W4A8_ERR_TIMEOUT, zero the workspace again.  Everything else in it is
+ * scratch between calls.
  */
 size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
@@ -131,8 +138,11 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   y          output [M, N] bf16 bit patterns (uint16), row-major.
  *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
  * M <= 16 runs the decode kernel (a weight-streaming GEMV); larger M runs
- * the tensor-core GEMM.  Two calls sharing one workspace must be ordered on
- * the GPU (same stream, or synchronised).
+ * the tensor-core GEMM.  For one token with K <= 15872 a single kernel
+ * rotates, quantises and applies the layer (every CTA quantises the token
+ * itself, with the activation kernel's arithmetic); otherwise the call is
+ * w4a8_linear_prepare followed by w4a8_linear_run.  Two calls sharing one
+ * workspace must be ordered on the GPU (same stream, or synchronised).
  * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA.
  */
 w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K,
@@ -179,7 +189,8 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
  * capture.  All calls on a device share the one array and leave their
  * scratch in it: calls whose work overlaps on the GPU (different streams
  * without ordering, or other host threads) race and give wrong results, so
- * order them.  What must start at zero is cleared by each call.
+ * order them.  What must start at zero is cleared by each call (it always
+ * runs the activation kernel and then the decode kernel, one token too).
  *   x, packed, y  as for w4a8_linear (device pointers owned by the caller).
  * Limits: M <= 16 (larger M returns W4A8_ERR_SHAPE); any shape needing more
  * scratch than the array holds returns W4A8_ERR_WORKSPACE (no accepted

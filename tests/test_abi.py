@@ -39,12 +39,16 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_packed_bytes_layout_arithmetic(lib):
+    # codebook (256) | row scales (4 N, padded to 256) | 32-row blocks of 0.5625 B per weight
+    def expect(n, k):
+        rows = -(-n // 32) * 32
+        body = rows * k // 2 + rows * k // 16
+        return 256 + -(-4 * n // 256) * 256 + -(-body // 256) * 256
     n, k = 17408, 5120
-    idx = n * k // 2
-    srel = n * k // 16
-    sch = -(-4 * n // 256) * 256
-    assert lib.w4a8_packed_bytes(n, k) == 256 + sch + idx + srel
-    assert lib.w4a8_packed_bytes(16, 256) == 256 + 256 + 16 * 128 + 16 * 16
+    assert lib.w4a8_packed_bytes(n, k) == 256 + 4 * n + n * k // 2 + n * k // 16
+    assert lib.w4a8_packed_bytes(n, k) == expect(n, k)
+    assert lib.w4a8_packed_bytes(16, 256) == 256 + 256 + 32 * 128 + 32 * 16
+    assert lib.w4a8_packed_bytes(48, 768) == expect(48, 768)
 
 
 @pytest.mark.parametrize("n,k", [(0, 256), (8, 256), (24, 256), (16, 300), (16, 0), (16, 65536), (-16, 256)])

@@ -229,7 +229,7 @@ def test_linear_deterministic_and_workspace_reuse(lib, layer592, m):
     bits, _, _ = synth.activations(m, 768, synth.rng_for(8, m, "act"), 8)
     xt = bf16(bits)
     need = max(lib.linear_workspace_bytes(mm, 768, 592) for mm in (1, 5, 16, 300))
-    ws = torch.empty(need + 4096, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(need + 4096, dtype=torch.uint8, device="cuda")
     a = lib.linear(xt, packed, 592, workspace=ws).clone()
     # a different shape through the same workspace in between
     other, _, _ = synth.activations(5, 768, synth.rng_for(8, 99, "act"), 8)
@@ -261,7 +261,7 @@ def test_prepare_once_run_several_layers(lib, m):
     layers = [converted(n, k, 40 + i) for i in range(3)]
     bits, x, _ = synth.activations(m, k, synth.rng_for(9, m, "act"), 8)
     xt = bf16(bits)
-    ws = torch.empty(lib.linear_workspace_bytes(m, k, n), dtype=torch.uint8, device="cuda")
+    ws = lib.linear_workspace(m, k, n, "cuda")
     lib.linear_prepare(xt, n, ws)
     for c in layers:
         packed = pack(lib, c)
@@ -270,3 +270,25 @@ def test_prepare_once_run_several_layers(lib, m):
         assert torch.equal(y_run.view(torch.int16), y_ref.view(torch.int16))
         wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
         check_linear(y_run.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+@pytest.mark.parametrize("k", [5120, 15872, 16128])
+def test_one_token_single_kernel_equals_two_kernel_path(lib, k):
+    """For one token and K <= 15872, w4a8_linear is one kernel that rotates and
+    quantises the token itself; it must give the same bits as the activation
+    kernel followed by the decode kernel (K = 16128 takes that path anyway),
+    and match the oracle."""
+    n = 592
+    c = O.convert_weight(synth.weights(n, k, synth.rng_for(70, k, "weight")), sample_cap=2**16)
+    packed = pack(lib, c)
+    bits, x, _ = synth.activations(1, k, synth.rng_for(10, k, "act"), max(1, k // 100))
+    xt = bf16(bits)
+    y_one = lib.linear(xt, packed, n)
+    ws = lib.linear_workspace(1, k, n, "cuda")
+    lib.linear_prepare(xt, n, ws)
+    y_two = lib.linear_run(1, k, packed, n, ws)
+    assert torch.equal(y_one.view(torch.int16), y_two.view(torch.int16))
+    # and again through the same workspace (its split-K counters were left at zero)
+    assert torch.equal(lib.linear(xt, packed, n, workspace=ws).view(torch.int16), y_one.view(torch.int16))
+    wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+    check_linear(y_one.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)

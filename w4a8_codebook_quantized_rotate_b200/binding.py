@@ -133,6 +133,14 @@ def linear_workspace_bytes(m: int, k: int, n: int) -> int:
     return int(load_library().w4a8_linear_workspace_bytes(m, k, n))
 
 
+def linear_workspace(m: int, k: int, n: int, device) -> torch.Tensor:
+    """A zero-filled workspace for layers of shape (M, K, N) (zero before its first use)."""
+    need = linear_workspace_bytes(m, k, n)
+    if need == 0:
+        raise W4A8Error("w4a8_linear_workspace_bytes", 2)
+    return torch.zeros(need, dtype=torch.uint8, device=device)
+
+
 def linear(x: torch.Tensor, packed: torch.Tensor, n: int, workspace: torch.Tensor | None = None,
            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """bf16 x [M, K] and a packed [N, K] layer -> bf16 y [M, N]."""
@@ -144,7 +152,7 @@ def linear(x: torch.Tensor, packed: torch.Tensor, n: int, workspace: torch.Tenso
     if need == 0:
         raise W4A8Error("w4a8_linear_workspace_bytes", 2)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
     _cuda(workspace, torch.uint8, "workspace")
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)

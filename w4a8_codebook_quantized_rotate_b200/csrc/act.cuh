@@ -58,6 +58,37 @@ __device__ __forceinline__ void fwht8_in_lane(float (&v)[8]) {
   }
 }
 
+// Lane's 8 values of the rotated 256-block b of a bf16 row: positions
+// 256 b + 8 lane .. + 7.  Three butterfly stages inside the lane, five across
+// lanes (shuffles), then the exact 1/16.
+__device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ row, int b, int lane, float (&v)[8]) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8);
+  const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(wds[i] << 16);
+    v[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+  }
+  fwht8_in_lane(v);
+#pragma unroll
+  for (int bit = 1; bit < 32; bit <<= 1) {
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[i], bit);
+      v[i] = upper ? (p - v[i]) : (v[i] + p);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;  // 1/16, exact
+}
+
+// Per-token scale and code: s = amax / 127 (IEEE division), q = clamp(rint(v / s), -127, 127).
+__device__ __forceinline__ float quant_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
+__device__ __forceinline__ float quant_code(float v, float s) {
+  return s > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v, s)), -127.f), 127.f) : 0.f;
+}
+
 template <int OUT>
 __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                   void* __restrict__ out, float* __restrict__ s_x,
@@ -79,29 +110,10 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
   const int nblocks = K / kRotBlock;
   float amax = 0.f;
   for (int b = warp; b < nblocks; b += nwarps) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(x + int64_t(m) * K + b * kRotBlock + lane * 8);
-    const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
     float v[8];
+    rotate_block_lane(x + int64_t(m) * K, b, lane, v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(wds[i] << 16);
-      v[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
-    }
-    fwht8_in_lane(v);
-#pragma unroll
-    for (int bit = 1; bit < 32; bit <<= 1) {
-      const bool upper = (lane & bit) != 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float p = __shfl_xor_sync(0xffffffffu, v[i], bit);
-        v[i] = upper ? (p - v[i]) : (v[i] + p);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] *= 0.0625f;  // 1/16, exact
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
     float4* dst = reinterpret_cast<float4*>(xr + b * kRotBlock + lane * 8);
     dst[0] = make_float4(v[0], v[1], v[2], v[3]);
     dst[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -113,7 +125,7 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
   amax = warp_max[0];
 #pragma unroll
   for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, warp_max[i]);
-  const float s = __fdiv_rn(amax, 127.0f);
+  const float s = quant_scale(amax);
   if (threadIdx.x == 0) s_x[m] = s;
   // Quantise 8 consecutive values per thread per step.
   for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
@@ -123,7 +135,7 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
     float q[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      q[i] = s > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -127.f), 127.f) : 0.f;
+      q[i] = quant_code(v[i], s);
     }
     if constexpr (OUT == kActI8Row) {
       uint32_t lo = 0, hi = 0;

@@ -4,20 +4,28 @@
 // dequant, decode and prefill kernels).  All region offsets are multiples of
 // 256 bytes.
 //
-//   [cb]   16 fp32 codebook levels
-//   [sch]  N fp32 row scales
-//   [idx]  index plane, [tile = N/16][chunk = K/64][lane 32][16 bytes]
-//   [srel] group-scale plane, [tile][chunk][64 bytes]
+//   [cb]     16 fp32 codebook levels
+//   [sch]    N fp32 row scales
+//   [units]  [pair = ceil(N/32)][chunk = K/64][1152 bytes]
 //
-// A (tile, chunk) block covers 16 rows x 64 k.  Its 512 index bytes are laid
-// out in the register order of the mma.sync m16n8k16 A operand, so that a
-// lane's 16 bytes are exactly its A fragments for the chunk's four k16 steps:
-// lane = 4 g + t (g = lane / 4, t = lane % 4), byte j = 4 s + r (s = k16 step,
-// r = fragment register) holds the canonical byte (two 4-bit indices, even k
-// in the low nibble) of
+// A unit covers the 32 rows of a tile pair (tiles 2p and 2p+1, 16 rows
+// each) and 64 k.  Its 1152 bytes are
+//   [0, 512)      index bytes of tile 2p
+//   [512, 1024)   index bytes of tile 2p+1
+//   [1024, 1088)  group-scale bytes of tile 2p
+//   [1088, 1152)  group-scale bytes of tile 2p+1
+// (a missing last tile, when N/16 is odd, is zero).  A unit is contiguous,
+// and units lie in [pair][chunk] order, so any range of units is one
+// contiguous run of memory that a single bulk copy can move.
+//
+// A tile's 512 index bytes are laid out in the register order of the
+// mma.sync m16n8k16 A operand, so that a lane's 16 bytes are exactly its A
+// fragments for the chunk's four k16 steps: lane = 4 g + t (g = lane / 4,
+// t = lane % 4), byte j = 4 s + r (s = k16 step, r = fragment register)
+// holds the canonical byte (two 4-bit indices, even k in the low nibble) of
 //     row  16 tile + g + 8 (r & 1)
 //     k    64 chunk + 16 s + 2 (t + 4 (r >> 1)), and k + 1.
-// The chunk's 64 group-scale bytes are [g 8][s 4][h 2]:
+// A tile's 64 group-scale bytes are [g 8][s 4][h 2]:
 //     byte 8 g + 2 s + h = s_rel[16 tile + g + 8 h][4 chunk + s].
 // One 16-bit half word then holds the pair (row g, row g + 8) of a k16 step,
 // which is the pair a lane needs to scale its accumulator fragment.
@@ -36,16 +44,17 @@ constexpr int kRotBlock = 256;
 constexpr int kGroup = 16;
 constexpr int kTileRows = 16;     // rows per (tile, chunk) block
 constexpr int kChunkK = 64;       // k per (tile, chunk) block
-constexpr int kChunkIdxBytes = 512;
-constexpr int kChunkSrelBytes = 64;
+constexpr int kChunkIdxBytes = 512;     // one tile's index bytes per chunk
+constexpr int kChunkSrelBytes = 64;     // one tile's group-scale bytes per chunk
+constexpr int kUnitBytes = 2 * kChunkIdxBytes + 2 * kChunkSrelBytes;  // 1152
 constexpr int kMaxK = 32768;
 
 // Device-side error word values (bit flags).
 constexpr unsigned kErrTimeout = 1u;
 
 struct PackedLayout {
-  int64_t N, K, tiles, chunks;
-  size_t off_cb, off_sch, off_idx, off_srel, total;
+  int64_t N, K, tiles, pairs, chunks;
+  size_t off_cb, off_sch, off_units, total;
 };
 
 __host__ __device__ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -55,13 +64,25 @@ __host__ __device__ inline PackedLayout packed_layout(int64_t N, int64_t K) {
   L.N = N;
   L.K = K;
   L.tiles = N / kTileRows;
+  L.pairs = (L.tiles + 1) / 2;
   L.chunks = K / kChunkK;
   L.off_cb = 0;
   L.off_sch = 256;
-  L.off_idx = L.off_sch + round_up(size_t(N) * 4, 256);
-  L.off_srel = L.off_idx + size_t(L.tiles) * L.chunks * kChunkIdxBytes;
-  L.total = round_up(L.off_srel + size_t(L.tiles) * L.chunks * kChunkSrelBytes, 256);
+  L.off_units = L.off_sch + round_up(size_t(N) * 4, 256);
+  L.total = round_up(L.off_units + size_t(L.pairs) * L.chunks * kUnitBytes, 256);
   return L;
+}
+
+// Byte offsets, within the units region, of tile `tile`'s index bytes and
+// group-scale bytes for chunk `chunk`.
+__host__ __device__ inline size_t unit_offset(int64_t pair, int64_t chunk, int64_t chunks) {
+  return size_t(pair * chunks + chunk) * kUnitBytes;
+}
+__host__ __device__ inline size_t tile_idx_offset(int64_t tile, int64_t chunk, int64_t chunks) {
+  return unit_offset(tile >> 1, chunk, chunks) + size_t(tile & 1) * kChunkIdxBytes;
+}
+__host__ __device__ inline size_t tile_srel_offset(int64_t tile, int64_t chunk, int64_t chunks) {
+  return unit_offset(tile >> 1, chunk, chunks) + 2 * kChunkIdxBytes + size_t(tile & 1) * kChunkSrelBytes;
 }
 
 // ---------------------------------------------------------------- small device helpers
@@ -159,6 +180,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const void* desc,
       "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_dst),
       "l"(desc), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple
+// of 16), completing `bytes` on the mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

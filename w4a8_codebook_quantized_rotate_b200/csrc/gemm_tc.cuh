@@ -41,8 +41,7 @@ constexpr uint32_t kTcACol = 256;     // A stages: columns [256, 384)
 constexpr size_t kTcSmemBytes = 1024 + 65536 + 65536 + size_t(kTcStagesB) * kTcStageBBytes;
 
 struct TcParams {
-  const uint8_t* idx;
-  const uint8_t* srel;
+  const uint8_t* units;   // unit region of the packed layer
   const float* sch;
   const float* cb;
   const float* s_x;
@@ -100,11 +99,10 @@ struct ExpStage {
 
 __device__ __forceinline__ void exp_load(ExpStage& e, const TcParams& p, int tile, int kb, int g, bool valid) {
   if (valid && kb < p.C) {
-    const size_t blk = size_t(tile) * p.C + kb;
-    const uint8_t* src = p.idx + blk * kChunkIdxBytes + size_t(4 * g) * 16;
+    const uint8_t* src = p.units + tile_idx_offset(tile, kb, p.C) + size_t(4 * g) * 16;
 #pragma unroll
     for (int t = 0; t < 4; ++t) e.seg[t] = __ldg(reinterpret_cast<const uint4*>(src) + t);
-    e.sr = __ldg(reinterpret_cast<const uint2*>(p.srel + blk * kChunkSrelBytes + g * 8));
+    e.sr = __ldg(reinterpret_cast<const uint2*>(p.units + tile_srel_offset(tile, kb, p.C) + g * 8));
   } else {
 #pragma unroll
     for (int t = 0; t < 4; ++t) e.seg[t] = make_uint4(0, 0, 0, 0);
@@ -260,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < 32; ++c) v[c] = 0u;
           }
           exp_load(es[i], p, tile, kb + 2 * PF, g, valid);
-          // lane 0 polls; the verdict is made warp-uniform before the
+          // lane 0 polls; the outcome is made warp-uniform before the
           // .sync.aligned TMEM store
           int w_ok = lane == 0 ? int(tc_wait(&sh->a_empty[sa], ((kb / kTcStagesA) & 1) ^ 1, sh, p.err)) : 0;
           ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;

@@ -29,6 +29,7 @@
 // adds those and writes y.
 #pragma once
 
+#include "act.cuh"
 #include "common.cuh"
 
 namespace w4a8 {
@@ -39,10 +40,15 @@ constexpr int kDecTG = 2;                          // tiles (16 rows each) per u
 constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
 constexpr int kDecMaxWarps = kDecMaxCtas * kDecWarps;
 constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
+constexpr int kDecSchRows = 1024;                  // row scales staged in shared memory per CTA
+// Units in flight per warp (register ring depth) per variant.
+constexpr int kDecDepthSingle = 3;                 // one token
+constexpr int kDecDepth1 = 3;                      // 2..8 tokens
+constexpr int kDecDepth2 = 2;                      // 9..16 tokens
 
 struct DecodeParams {
-  const uint8_t* idx;    // index plane
-  const uint8_t* srel;   // group-scale plane
+  const uint16_t* x;     // one token's bf16 activations [K] (the kernel that rotates and quantises them itself)
+  const uint8_t* units;  // unit region of the packed layer (contiguous 1152-byte units, [pair][chunk])
   const float* sch;      // [N]
   const float* cb;       // [16]
   const uint4* xfrag;    // activations in B-fragment order, [C][NB][32][2] uint4
@@ -51,7 +57,8 @@ struct DecodeParams {
   float* slots;          // [2 * CTAs][kDecTG * 16][M]: per-CTA partials of pairs shared with other CTAs
   unsigned* counters;    // [P]
   unsigned* err;
-  int M, N, C, T, P, W, U;
+  int M, N, K, C, T, P, W, U;
+  int R, Rm;  // U / W and U % W: warp w's first unit is w R + floor(w Rm / W)
 };
 
 // Floats of one partial (a tile pair, the first M tokens).
@@ -60,25 +67,25 @@ __host__ __device__ inline int dec_slot_floats(int m) { return kDecTG * 16 * m; 
 // Dynamic shared memory of a launch: table (+ alignment room), one token's
 // activations, and the CTA's per-warp partials.
 __host__ __device__ inline size_t dec_smem_bytes(int m, int k, bool single) {
-  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(kDecWarps) * 2 * dec_slot_floats(m) * 4;
+  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(kDecWarps) * 2 * dec_slot_floats(m) * 4 +
+         kDecSchRows * 4 + 64 + 128 + 64;
 }
 
-// Ranges: warp w holds units [floor(w U / W), floor((w+1) U / W)).
-__device__ __forceinline__ int dec_range_begin(int w, int U, int W) { return int(int64_t(w) * U / W); }
-__device__ __forceinline__ int dec_warp_of(int u, int U, int W) { return int((int64_t(u + 1) * W - 1) / U); }
+// Largest K of the kernel that rotates and quantises its token itself: the
+// fp32 rotated row is staged below the 64 KiB-aligned table, in the first
+// 64 KiB of the CTA's shared window less the 1 KiB the system reserves.
+constexpr int kDecFusedMaxK = 15872;
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+// Ranges: warp w holds units [floor(w U / W), floor((w+1) U / W)); in 32-bit
+// arithmetic as w R + floor(w Rm / W) (w Rm < W^2 < 2^32).  w may be W.
+__device__ __forceinline__ int dec_begin(int w, const DecodeParams& p) {
+  return w * p.R + int((unsigned(w) * unsigned(p.Rm)) / unsigned(p.W));
 }
-__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
+// CTA c holds warps [16 c, 16 c + 16) (clipped at W).
+__device__ __forceinline__ int dec_cta_begin(int c, const DecodeParams& p) {
+  return dec_begin(min(c * kDecWarps, p.W), p);
 }
+
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -106,14 +113,6 @@ __device__ __forceinline__ void mma_16816z(float (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%10, %10, %10, %10};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
-}
-
 // Per-unit registers: index bytes and group scales of the two tiles, and (for
 // more than one token) the B fragments of the unit's chunk.
 template <int NB, bool SINGLE>
@@ -123,46 +122,36 @@ struct DecStage {
   uint4 x[SINGLE ? 1 : NB][2];
 };
 
-// Where the next unit to prefetch lies.  The second tile of a pair sits
-// C blocks after the first; for an odd tile count the missing last tile
-// re-reads the first (its results are never stored).
-struct DecCursor {
-  const uint8_t* idx;   // this lane's 16 bytes of tile 0
-  const uint8_t* srel;  // this lane's 8 scale bytes of tile 0
-  uint32_t idx1, srel1; // byte offsets of tile 1
-  int pair, c;
-};
-
-__device__ __forceinline__ void dec_cursor_pair(DecCursor& q, const DecodeParams& p) {
-  const bool two = q.pair * kDecTG + 1 < p.T;
-  q.idx1 = two ? uint32_t(p.C) * kChunkIdxBytes : 0u;
-  q.srel1 = two ? uint32_t(p.C) * kChunkSrelBytes : 0u;
+__device__ __forceinline__ uint4 ld_stream_v4(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_stream_v2(const uint8_t* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
 }
 
-__device__ __forceinline__ void dec_cursor_advance(DecCursor& q, const DecodeParams& p) {
-  q.idx += kChunkIdxBytes;
-  q.srel += kChunkSrelBytes;
-  if (++q.c == p.C) {
-    q.c = 0;
-    ++q.pair;
-    q.idx += size_t(p.C) * kChunkIdxBytes;  // skip the previous pair's second tile
-    q.srel += size_t(p.C) * kChunkSrelBytes;
-    dec_cursor_pair(q, p);
-  }
+// A lane's index words and scale codes of one unit: wp points at the lane's
+// 16 index bytes of tile 0 in the unit, sp at its 8 scale bytes of tile 0.
+template <int NB, bool SINGLE>
+__device__ __forceinline__ void dec_load_w(DecStage<NB, SINGLE>& st, const uint8_t* wp, const uint8_t* sp) {
+  st.w[0] = ld_stream_v4(wp);
+  st.w[1] = ld_stream_v4(wp + kChunkIdxBytes);
+  st.s[0] = ld_stream_v2(sp);
+  st.s[1] = ld_stream_v2(sp + kChunkSrelBytes);
 }
 
 template <int NB, bool SINGLE>
-__device__ __forceinline__ void dec_load(DecStage<NB, SINGLE>& st, const DecCursor& q, const DecodeParams& p,
-                                         int lane) {
-  st.w[0] = ld_stream_v4(q.idx);
-  st.w[1] = ld_stream_v4(q.idx + q.idx1);
-  st.s[0] = ld_stream_v2(q.srel);
-  st.s[1] = ld_stream_v2(q.srel + q.srel1);
+__device__ __forceinline__ void dec_load_x(DecStage<NB, SINGLE>& st, const DecodeParams& p, int c, int lane) {
   if constexpr (!SINGLE) {
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
       if ((lane >> 2) + 8 * j < p.M) {
-        const uint4* src = p.xfrag + (size_t(q.c * NB + j) * 32 + lane) * 2;
+        const uint4* src = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
         st.x[j][0] = __ldg(src);
         st.x[j][1] = __ldg(src + 1);
       } else {
@@ -238,23 +227,42 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, floa
 
 // acc element e of (tile i, block j) is row 16 (2 pair + i) + g + 8 (e >> 1),
 // token 8 j + 2 t + (e & 1).
+// Row scales of the CTA's first kDecSchRows rows (from row0) and the tokens'
+// s_x sit in shared memory; rows past those are read from global memory.
+struct DecEpi {
+  uint32_t sch;  // shared address of row scales [row0, row0 + kDecSchRows)
+  uint32_t sx;   // shared address of s_x[0..M)
+  int row0;
+};
+
 template <int NB>
 __device__ __forceinline__ void dec_epilogue(const float (&acc)[kDecTG][NB][4], const DecodeParams& p, int pair,
-                                             int lane) {
+                                             int lane, const DecEpi& ep) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int i = 0; i < kDecTG; ++i) {
     const int tile = pair * kDecTG + i;
     if (tile >= p.T) continue;
 #pragma unroll
-    for (int j = 0; j < NB; ++j) {
+    for (int h = 0; h < 2; ++h) {
+      const int row = tile * 16 + g + 8 * h;
+      const int rr = row - ep.row0;
+      float sc;
+      if (rr < kDecSchRows)
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(ep.sch + uint32_t(rr) * 4u));
+      else
+        sc = __ldg(p.sch + row);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = tile * 16 + g + 8 * (e >> 1);
-        const int tok = 8 * j + 2 * t + (e & 1);
-        if (tok < p.M) {
-          const float v = acc[i][j][e] * p.sch[row] * p.s_x[tok];
-          p.y[size_t(tok) * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+      for (int j = 0; j < NB; ++j) {
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int tok = 8 * j + 2 * t + e2;
+          if (tok < p.M) {
+            float sx;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sx) : "r"(ep.sx + uint32_t(tok) * 4u));
+            const float v = acc[i][j][2 * h + e2] * sc * sx;
+            p.y[size_t(tok) * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          }
         }
       }
     }
@@ -311,8 +319,26 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 }
 
-template <int NB, int D, bool SINGLE>
+// ---------------------------------------------------------------------------
+// Work split ("stream-K"): the P * C units, in the order they lie in memory,
+// are cut into W equal ranges, one per warp; a CTA's 16 warps hold 16
+// consecutive ranges, so each warp streams one contiguous byte range.  A
+// warp keeps D units in flight in registers (a ring refilled right after
+// each unit is computed).  A warp that covers a whole tile pair writes y
+// directly.  A pair split between warps is reduced in two levels, both in a
+// fixed order (the result is deterministic): the warps of a CTA leave their
+// partials in shared memory and one warp adds them after a CTA barrier; a
+// pair that also crosses into another CTA leaves one partial per CTA in the
+// workspace, and the last CTA to finish it (an atomic counter, no waiting)
+// adds those and writes y.
+//
+// FUSED (one token): the kernel also does the activation step: every CTA
+// rotates the bf16 row and quantises it to int8 (the activation kernel's
+// arithmetic, so the codes and s_x are the same bits), staging the rotated
+// row in fp32 below the table.  One launch then makes the whole layer.
+template <int NB, int D, bool SINGLE, bool FUSED = false>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
+  static_assert(!FUSED || SINGLE, "the fused activation step handles one token");
   extern __shared__ __align__(16) uint8_t dec_smem[];
   // The next kernel may launch now: it streams its own weights and waits for
   // this grid's completion before it touches anything this grid writes.
@@ -322,37 +348,53 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   const uint32_t xs = lut + 65536u;                   // one token: x staged here (2 K bytes)
   const uint32_t parts = xs + (SINGLE ? uint32_t(p.C) * 128u : 0u);  // [warp][2] partials
   const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
-  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const int w = blockIdx.x * kDecWarps + wl;
-  const bool active = w < p.W;
-  const int u0 = active ? dec_range_begin(w, p.U, p.W) : 0;
-  const int u1 = active ? dec_range_begin(w + 1, p.U, p.W) : 0;
-  const int n_units = u1 - u0;
-
-  DecCursor q;
-  q.pair = u0 / p.C;
-  q.c = u0 - q.pair * p.C;
-  {
-    const size_t blk = size_t(q.pair) * kDecTG * p.C + q.c;
-    q.idx = p.idx + blk * kChunkIdxBytes + lane * 16;
-    q.srel = p.srel + blk * kChunkSrelBytes + (lane >> 2) * 8;
+  const uint32_t sch_s = parts + uint32_t(kDecWarps * 2) * part_bytes;  // row scales
+  const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
+  const uint32_t wbeg_s = sx_s + 64;                                      // warp range starts [17]
+  const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
+  const uint32_t rot_s = (base + 15u) & ~15u;                             // FUSED: rotated row [K] fp32
+  if (FUSED && rot_s + uint32_t(p.K) * 4u > lut) {  // the launch does not leave room below the table
+    if (threadIdx.x == 0) record_error(p.err, kErrTimeout);
+    return;
   }
-  dec_cursor_pair(q, p);
-  const int first_pair = q.pair;
-  const int first_c = q.c;
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int cta_w0 = blockIdx.x * kDecWarps;
+  const int w = cta_w0 + wl;
+  const int u0 = dec_begin(min(w, p.W), p);
+  const int u1 = dec_begin(min(w + 1, p.W), p);
+  const int n_units = u1 - u0;
+  const int first_pair = u0 / p.C;
+  const int first_c = u0 - first_pair * p.C;
+
+  // This lane's index bytes and scale bytes in unit u0; every later unit is
+  // kUnitBytes further on.
+  const uint8_t* wp = p.units + size_t(u0) * kUnitBytes + lane * 16;
+  const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8;
 
   DecStage<NB, SINGLE> st[D];
   // Weights do not depend on the previous kernel: start streaming them first.
   // (x for more than one token comes from it, so it is loaded after the wait.)
 #pragma unroll
-  for (int d = 0; d < D; ++d) {
-    if (d < n_units) {
-      st[d].w[0] = ld_stream_v4(q.idx);
-      st[d].w[1] = ld_stream_v4(q.idx + q.idx1);
-      st[d].s[0] = ld_stream_v2(q.srel);
-      st[d].s[1] = ld_stream_v2(q.srel + q.srel1);
-      dec_cursor_advance(q, p);
-    }
+  for (int d = 0; d < D; ++d)
+    if (d < n_units) dec_load_w<NB, SINGLE>(st[d], wp + d * kUnitBytes, sp + d * kUnitBytes);
+  wp += D * kUnitBytes;
+  sp += D * kUnitBytes;
+
+  // The CTA's range, its warps' range starts and its rows' scales (all
+  // independent of the previous kernel).
+  const int v0 = dec_cta_begin(blockIdx.x, p), v1 = dec_cta_begin(blockIdx.x + 1, p);
+  if (lane == 0) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(wl) * 4u), "r"(u0));
+    if (wl == kDecWarps - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + 64u), "r"(v1));
+  }
+  DecEpi ep;
+  ep.sch = sch_s;
+  ep.sx = sx_s;
+  ep.row0 = (v0 / p.C) * (kDecTG * 16);
+  {
+    const int rows = min(kDecSchRows, min(p.N, (v1 > v0 ? (v1 - 1) / p.C + 1 : 0) * kDecTG * 16) - ep.row0);
+    for (int i = threadIdx.x; i < rows; i += kDecThreads)
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(sch_s + uint32_t(i) * 4u), "f"(__ldg(p.sch + ep.row0 + i)));
   }
   // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
   {
@@ -366,34 +408,65 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     }
   }
   pdl_wait();  // activations, scales and counters come from the previous kernel
-  if constexpr (SINGLE) {
-    // token 0's B fragments: per chunk, lanes t = 0..3 of the fragment layout (128 bytes)
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.xfrag);
-    for (int e = threadIdx.x; e < p.C * 8; e += kDecThreads) {
-      const int c = e >> 3, qq = e & 7;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + size_t(c) * 1024 + qq * 16));
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + uint32_t(c) * 128u + uint32_t(qq) * 16u),
-                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+  int cx = first_c;  // chunk of the next x fragment to load (more than one token)
+  if constexpr (FUSED) {
+    // Rotate the row (warp per 256-block) and find its absmax.
+    float amax = 0.f;
+    for (int b = wl; b < p.K / kRotBlock; b += kDecWarps) {
+      float v[8];
+      rotate_block_lane(p.x, b, lane, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      const uint32_t dst = rot_s + uint32_t(b * kRotBlock + lane * 8) * 4u;
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+                   "f"(v[7]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(red_s + uint32_t(wl) * 4u), "f"(amax));
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kDecWarps; ++i) {
+      float m;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(m) : "r"(red_s + uint32_t(i) * 4u));
+      amax = fmaxf(amax, m);
+    }
+    const float s = quant_scale(amax);
+    if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s), "f"(s));
+    // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
+    // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4.
+    for (int k0 = threadIdx.x * 8; k0 < p.K; k0 += kDecThreads * 8) {
+      float v[8];
+      const uint32_t src = rot_s + uint32_t(k0) * 4u;
+      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(src));
+      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(src + 16u));
+      const uint32_t dst = xs + uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const __half2 h = __floats2half2_rn(quant_code(v[2 * t], s), quant_code(v[2 * t + 1], s));
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + uint32_t(t) * 32u), "r"(*reinterpret_cast<const uint32_t*>(&h)));
+      }
     }
   } else {
-    int c = first_c;
+    if (threadIdx.x < p.M)
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + threadIdx.x * 4u), "f"(p.s_x[threadIdx.x]));
+    if constexpr (SINGLE) {
+      // token 0's B fragments: per chunk, lanes t = 0..3 of the fragment layout (128 bytes)
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(p.xfrag);
+      for (int e = threadIdx.x; e < p.C * 8; e += kDecThreads) {
+        const int c = e >> 3, qq = e & 7;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + size_t(c) * 1024 + qq * 16));
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + uint32_t(c) * 128u + uint32_t(qq) * 16u),
+                     "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+      }
+    } else {
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      if (d < n_units) {
-        if constexpr (!SINGLE) {
-#pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            if ((lane >> 2) + 8 * j < p.M) {
-              const uint4* srcx = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
-              st[d].x[j][0] = __ldg(srcx);
-              st[d].x[j][1] = __ldg(srcx + 1);
-            } else {
-              st[d].x[j][0] = make_uint4(0, 0, 0, 0);
-              st[d].x[j][1] = make_uint4(0, 0, 0, 0);
-            }
-          }
+      for (int d = 0; d < D; ++d) {
+        if (d < n_units) {
+          dec_load_x<NB, SINGLE>(st[d], p, cx, lane);
+          if (++cx == p.C) cx = 0;
         }
-        if (++c == p.C) c = 0;
       }
     }
   }
@@ -408,13 +481,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   // else park the partial in shared memory (slot 0: the warp's first pair).
   auto close_pair = [&](int c_last) {
     if (c_first == 0 && c_last == p.C - 1) {
-      dec_epilogue<NB>(acc, p, cur_pair, lane);
+      dec_epilogue<NB>(acc, p, cur_pair, lane, ep);
     } else {
       const uint32_t slot = parts + uint32_t(wl * 2 + (cur_pair == first_pair ? 0 : 1)) * part_bytes;
       dec_partial_store_smem<NB>(acc, slot, p.M, lane);
     }
   };
-
   auto unit_done = [&]() {
     if (++cur_c == p.C) {
       close_pair(p.C - 1);
@@ -424,16 +496,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       c_first = 0;
     }
   };
+  auto refill = [&](DecStage<NB, SINGLE>& s, int off_units) {
+    dec_load_w<NB, SINGLE>(s, wp + off_units * kUnitBytes, sp + off_units * kUnitBytes);
+    if constexpr (!SINGLE) {
+      dec_load_x<NB, SINGLE>(s, p, cx, lane);
+      if (++cx == p.C) cx = 0;
+    }
+  };
   int ub = 0;
   // Full rounds: every stage computes and refills.
   for (; ub + 2 * D <= n_units; ub += D) {
 #pragma unroll
     for (int d = 0; d < D; ++d) {
       dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
-      dec_load<NB, SINGLE>(st[d], q, p, lane);
-      dec_cursor_advance(q, p);
+      refill(st[d], d);
       unit_done();
     }
+    wp += D * kUnitBytes;
+    sp += D * kUnitBytes;
   }
   // Tail: fewer than 2 D units left.
 #pragma unroll
@@ -441,10 +521,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     const int d = d2 % D;
     if (ub + d2 < n_units) {
       dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
-      if (ub + d2 + D < n_units) {
-        dec_load<NB, SINGLE>(st[d], q, p, lane);
-        dec_cursor_advance(q, p);
-      }
+      if (ub + d2 + D < n_units) refill(st[d], d2);
       unit_done();
     }
   }
@@ -452,33 +529,37 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   __syncthreads();
 
   // ---- level 2: pairs split between warps, reduced by one warp of the CTA
-  const int cta_w0 = blockIdx.x * kDecWarps;
-  const int cta_w1 = min(cta_w0 + kDecWarps, p.W);  // exclusive
-  if (cta_w0 >= cta_w1) return;
-  const int v0 = dec_range_begin(cta_w0, p.U, p.W);
-  const int v1 = dec_range_begin(cta_w1, p.U, p.W);
+  if (v0 >= v1) return;
+  auto wbeg = [&](int i) -> int {
+    int v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(wbeg_s + uint32_t(i) * 4u));
+    return v;
+  };
   const int pair_lo = v0 / p.C, pair_hi = (v1 - 1) / p.C;
   for (int pr = pair_lo + wl; pr <= pair_hi; pr += kDecWarps) {
-    const int wf = dec_warp_of(pr * p.C, p.U, p.W);            // first warp holding this pair
-    const int wlst = dec_warp_of(pr * p.C + p.C - 1, p.U, p.W);  // last warp holding it
-    if (wf == wlst) continue;                                    // one warp held all of it: done
-    const int a = max(wf, cta_w0), z = min(wlst, cta_w1 - 1);     // this CTA's contributors
+    const int q0 = pr * p.C, q1 = q0 + p.C;  // the pair's units [q0, q1)
+    bool whole = false;                       // one warp held all of it (and wrote y)
+    for (int ww = 0; ww < kDecWarps; ++ww) whole = whole || (wbeg(ww) <= q0 && wbeg(ww + 1) >= q1);
+    if (whole) continue;
     dec_zero<NB>(acc);
-    for (int ww = a; ww <= z; ++ww) {
-      const int first_of_ww = dec_range_begin(ww, p.U, p.W) / p.C;
-      const uint32_t slot = parts + uint32_t((ww - cta_w0) * 2 + (pr == first_of_ww ? 0 : 1)) * part_bytes;
-      dec_partial_add_smem<NB>(acc, slot, p.M, lane);
+    for (int ww = 0; ww < kDecWarps; ++ww) {
+      const int b0 = wbeg(ww), b1 = wbeg(ww + 1);
+      if (b0 < q1 && b1 > q0 && b0 < b1) {  // warp ww holds some of it
+        const uint32_t slot = parts + uint32_t(ww * 2 + (b0 >= q0 ? 0 : 1)) * part_bytes;
+        dec_partial_add_smem<NB>(acc, slot, p.M, lane);
+      }
     }
-    const int cf = dec_warp_of(pr * p.C, p.U, p.W) / kDecWarps;             // first CTA holding the pair
-    const int cl = dec_warp_of(pr * p.C + p.C - 1, p.U, p.W) / kDecWarps;   // last CTA holding it
-    if (cf == cl) {
-      dec_epilogue<NB>(acc, p, pr, lane);
+    if (q0 >= v0 && q1 <= v1) {  // inside this CTA
+      dec_epilogue<NB>(acc, p, pr, lane, ep);
       continue;
     }
-    // ---- level 3: the pair spans CTAs; park this CTA's partial in the workspace
+    // ---- level 3: the pair spans CTAs cf..cl; park this CTA's partial in the workspace
+    int cf = blockIdx.x, cl = blockIdx.x;
+    while (cf > 0 && dec_cta_begin(cf, p) > q0) --cf;
+    while (dec_cta_begin(cl + 1, p) < q1) ++cl;
     const int sf = dec_slot_floats(p.M);
     const int g = lane >> 2, t = lane & 3;
-    float* mine = p.slots + size_t(blockIdx.x * 2 + (pr == pair_lo ? 0 : 1)) * sf;
+    float* mine = p.slots + size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf;
 #pragma unroll
     for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
@@ -496,7 +577,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     if (old != unsigned(cl - cf)) continue;  // another CTA finishes this pair
     __threadfence();
     // Sum the CTAs' partials in CTA order; all loads are independent.
-    constexpr int kMaxCtaParts = 8 / NB;
+    constexpr int kMaxCtaParts = 4 / NB;
     dec_zero<NB>(acc);
     for (int c0 = cf; c0 <= cl; c0 += kMaxCtaParts) {
       float v[kMaxCtaParts][kDecTG][NB][4];
@@ -504,8 +585,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       for (int r = 0; r < kMaxCtaParts; ++r) {
         const int cc = c0 + r;
         const bool have = cc <= cl;
-        const int first_of_cc = dec_range_begin(cc * kDecWarps, p.U, p.W) / p.C;
-        const float* src = p.slots + size_t(cc * 2 + (pr == first_of_cc ? 0 : 1)) * sf;
+        const float* src = p.slots + size_t(cc * 2 + (have && dec_cta_begin(cc, p) >= q0 ? 0 : 1)) * sf;
 #pragma unroll
         for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
@@ -526,7 +606,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
             for (int e = 0; e < 4; ++e) acc[i][j][e] += v[r][i][j][e];
     }
     if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
-    dec_epilogue<NB>(acc, p, pr, lane);
+    dec_epilogue<NB>(acc, p, pr, lane, ep);
   }
 }
 

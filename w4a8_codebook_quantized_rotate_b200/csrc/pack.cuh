@@ -10,46 +10,54 @@
 
 namespace w4a8 {
 
-// One thread per (tile, chunk, lane): gathers the lane's 16 index bytes from
-// the canonical [N, K/2] plane; lanes 0..15 also move 4 group-scale bytes.
+// One thread per (tile, chunk, lane) over 2 * pairs tiles: gathers the
+// lane's 16 index bytes from the canonical [N, K/2] plane; lanes 0..15 also
+// move 4 group-scale bytes.  The missing last tile of an odd tile count is
+// written as zeros.
 __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ idx,
                                                    const uint8_t* __restrict__ s_rel, int64_t N, int64_t K,
-                                                   uint8_t* __restrict__ idx_plane,
-                                                   uint8_t* __restrict__ srel_plane) {
+                                                   uint8_t* __restrict__ units) {
   const int64_t chunks = K / kChunkK;
   const int64_t tiles = N / kTileRows;
+  const int64_t tiles_padded = 2 * ((tiles + 1) / 2);
   const int64_t gtid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t block = gtid >> 5;  // (tile, chunk) block
   const int lane = int(gtid & 31);
-  if (block >= tiles * chunks) return;
+  if (block >= tiles_padded * chunks) return;
   const int64_t tile = block / chunks;
   const int64_t chunk = block - tile * chunks;
+  const bool real = tile < tiles;
   const int g = lane >> 2, t = lane & 3;
   const int64_t row_bytes = K / 2;
-  uint32_t w[4];
+  uint32_t w[4] = {0, 0, 0, 0};
+  if (real) {
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    uint32_t v = 0;
+    for (int s = 0; s < 4; ++s) {
+      uint32_t v = 0;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int64_t row = tile * kTileRows + g + 8 * (r & 1);
-      const int64_t col = chunk * 32 + 8 * s + t + 4 * (r >> 1);
-      v |= uint32_t(idx[row * row_bytes + col]) << (8 * r);
+      for (int r = 0; r < 4; ++r) {
+        const int64_t row = tile * kTileRows + g + 8 * (r & 1);
+        const int64_t col = chunk * 32 + 8 * s + t + 4 * (r >> 1);
+        v |= uint32_t(idx[row * row_bytes + col]) << (8 * r);
+      }
+      w[s] = v;
     }
-    w[s] = v;
   }
-  *reinterpret_cast<uint4*>(idx_plane + (block * 32 + lane) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(units + tile_idx_offset(tile, chunk, chunks) + lane * 16) =
+      make_uint4(w[0], w[1], w[2], w[3]);
   if (lane < 16) {
     const int64_t row_groups = K / kGroup;
     uint32_t v = 0;
+    if (real) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int q = lane * 4 + e;  // byte 8 g + 2 s + h of the chunk's 64
-      const int gg = q >> 3, s = (q >> 1) & 3, h = q & 1;
-      const int64_t row = tile * kTileRows + gg + 8 * h;
-      v |= uint32_t(s_rel[row * row_groups + chunk * 4 + s]) << (8 * e);
+      for (int e = 0; e < 4; ++e) {
+        const int q = lane * 4 + e;  // byte 8 g + 2 s + h of the tile's 64
+        const int gg = q >> 3, s = (q >> 1) & 3, h = q & 1;
+        const int64_t row = tile * kTileRows + gg + 8 * h;
+        v |= uint32_t(s_rel[row * row_groups + chunk * 4 + s]) << (8 * e);
+      }
     }
-    *reinterpret_cast<uint32_t*>(srel_plane + block * kChunkSrelBytes + lane * 4) = v;
+    *reinterpret_cast<uint32_t*>(units + tile_srel_offset(tile, chunk, chunks) + lane * 4) = v;
   }
 }
 
@@ -63,8 +71,7 @@ __global__ void copy_scales_kernel(const float* __restrict__ s_channel, const fl
 // One warp per (tile, chunk) block.  Each lane rebuilds its 32 weights and
 // writes them as float2 pairs; across the warp every 32-byte sector of the
 // output rows is written whole.
-__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ idx_plane,
-                                                      const uint8_t* __restrict__ srel_plane,
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ units,
                                                       const float* __restrict__ sch, const float* __restrict__ cb,
                                                       int64_t N, int64_t K, float* __restrict__ w_hat) {
   __shared__ float cb_s[16];
@@ -78,8 +85,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   const int64_t tile = block / chunks;
   const int64_t chunk = block - tile * chunks;
   const int g = lane >> 2, t = lane & 3;
-  const uint4 wv = *reinterpret_cast<const uint4*>(idx_plane + (block * 32 + lane) * 16);
-  const uint2 sv = *reinterpret_cast<const uint2*>(srel_plane + block * kChunkSrelBytes + g * 8);
+  const uint4 wv = *reinterpret_cast<const uint4*>(units + tile_idx_offset(tile, chunk, chunks) + lane * 16);
+  const uint2 sv = *reinterpret_cast<const uint2*>(units + tile_srel_offset(tile, chunk, chunks) + g * 8);
   const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
   const float s_row[2] = {sch[tile * kTileRows + g], sch[tile * kTileRows + g + 8]};
 #pragma unroll

@@ -75,9 +75,11 @@ w4a8_status device_state(DeviceState** out) {
       if (allow_smem(rotate_quant_kernel<kActI8Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Frag>, size_t(kMaxK) * 4) != cudaSuccess ||
-          allow_smem(decode_kernel<1, 4, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
-          allow_smem(decode_kernel<1, 3, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
-          allow_smem(decode_kernel<2, 2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<1, kDecDepthSingle, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
+          allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kDecFusedMaxK, true)) !=
+              cudaSuccess ||
+          allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<2, kDecDepth2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
         return W4A8_ERR_CUDA;
     }
@@ -182,9 +184,8 @@ w4a8_status w4a8_pack_layout(const uint8_t* idx, const uint8_t* s_rel, const flo
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(packed);
-  const int64_t threads = L.tiles * L.chunks * 32;
-  pack_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(idx, s_rel, N, K, base + L.off_idx,
-                                                              base + L.off_srel);
+  const int64_t threads = 2 * L.pairs * L.chunks * 32;
+  pack_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(idx, s_rel, N, K, base + L.off_units);
   copy_scales_kernel<<<unsigned((N + 255) / 256), 256, 0, s>>>(s_channel, codebook, N,
                                                                 reinterpret_cast<float*>(base + L.off_sch),
                                                                 reinterpret_cast<float*>(base + L.off_cb));
@@ -201,7 +202,7 @@ w4a8_status w4a8_unpack_dequant(const void* packed, int64_t N, int64_t K, float*
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   const int64_t threads = L.tiles * L.chunks * 32;
   dequant_kernel<<<unsigned((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      base + L.off_idx, base + L.off_srel, reinterpret_cast<const float*>(base + L.off_sch),
+      base + L.off_units, reinterpret_cast<const float*>(base + L.off_sch),
       reinterpret_cast<const float*>(base + L.off_cb), N, K, w_hat);
   return launch_status();
 }
@@ -231,6 +232,48 @@ static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* wo
   *plan = linear_plan(M, K, N);
   if (workspace_bytes < plan->total) return W4A8_ERR_WORKSPACE;
   return device_state(d);
+}
+
+// Decode launch (M <= 16).  With x given (one token, K <= kDecFusedMaxK) the
+// kernel also rotates and quantises the token; otherwise it reads what
+// w4a8_linear_prepare left in the workspace.
+static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, int64_t M, int64_t K, int64_t N,
+                                 const uint8_t* pk, uint16_t* y, uint8_t* ws, cudaStream_t s, const uint16_t* x) {
+  const PackedLayout L = packed_layout(N, K);
+  DecodeParams p;
+  p.x = x;
+  p.units = pk + L.off_units;
+  p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
+  p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
+  p.xfrag = reinterpret_cast<const uint4*>(ws + plan.off_xq);
+  p.s_x = reinterpret_cast<const float*>(ws + plan.off_sx);
+  p.y = y;
+  p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
+  p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
+  p.err = d->err;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.C = plan.C;
+  p.T = plan.T;
+  p.P = plan.P;
+  p.U = plan.P * plan.C;
+  const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
+  p.W = p.U < warps_avail ? p.U : warps_avail;
+  p.R = p.U / p.W;
+  p.Rm = p.U % p.W;
+  const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
+  const size_t smem = dec_smem_bytes(int(M), int(K), M == 1);
+  cudaError_t e;
+  if (x)
+    e = launch_pdl(decode_kernel<1, kDecDepthSingle, true, true>, grid, dim3(kDecThreads), smem, s, p);
+  else if (plan.nb == 1 && M == 1)
+    e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
+  else if (plan.nb == 1)
+    e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(kDecThreads), smem, s, p);
+  else
+    e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(kDecThreads), smem, s, p);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
 w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
@@ -269,37 +312,7 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* s_x = reinterpret_cast<float*>(ws + plan.off_sx);
 
-  if (plan.decode) {
-    DecodeParams p;
-    p.idx = pk + L.off_idx;
-    p.srel = pk + L.off_srel;
-    p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
-    p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
-    p.xfrag = reinterpret_cast<const uint4*>(ws + plan.off_xq);
-    p.s_x = s_x;
-    p.y = y;
-    p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
-    p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
-    p.err = d->err;
-    p.M = int(M);
-    p.N = int(N);
-    p.C = plan.C;
-    p.T = plan.T;
-    p.P = plan.P;
-    p.U = plan.P * plan.C;
-    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
-    p.W = p.U < warps_avail ? p.U : warps_avail;
-    const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
-    cudaError_t e;
-    const size_t smem = dec_smem_bytes(int(M), int(K), M == 1);
-    if (plan.nb == 1 && M == 1)
-      e = launch_pdl(decode_kernel<1, 4, true>, grid, dim3(kDecThreads), smem, s, p);
-    else if (plan.nb == 1)
-      e = launch_pdl(decode_kernel<1, 3, false>, grid, dim3(kDecThreads), smem, s, p);
-    else
-      e = launch_pdl(decode_kernel<2, 2, false>, grid, dim3(kDecThreads), smem, s, p);
-    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
-  }
+  if (plan.decode) return launch_decode(plan, d, M, K, N, pk, y, ws, s, nullptr);
 
   __half* xq = reinterpret_cast<__half*>(ws + plan.off_xq);
   EncodeTiledFn enc = encode_fn();
@@ -314,8 +327,7 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return W4A8_ERR_CUDA;
   TcParams p;
-  p.idx = pk + L.off_idx;
-  p.srel = pk + L.off_srel;
+  p.units = pk + L.off_units;
   p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
   p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
   p.s_x = s_x;
@@ -335,6 +347,14 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* pac
                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !packed || !y || !workspace) return W4A8_ERR_NULL;
   if (!aligned16(packed) || !aligned16(y)) return W4A8_ERR_ALIGN;
+  if (M == 1 && K <= kDecFusedMaxK) {  // one token: a single kernel makes the layer
+    if (!aligned16(x)) return W4A8_ERR_ALIGN;
+    LinearPlan plan;
+    DeviceState* d = nullptr;
+    if (w4a8_status st = linear_checks(M, K, N, workspace, workspace_bytes, &plan, &d); st != W4A8_OK) return st;
+    return launch_decode(plan, d, M, K, N, static_cast<const uint8_t*>(packed), y, static_cast<uint8_t*>(workspace),
+                         static_cast<cudaStream_t>(stream), x);
+  }
   w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
@@ -363,9 +383,11 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, c
     scratch = g_static_scratch_ptr[dev];
   }
   // The split-K counters the decode kernel needs at zero are cleared by the
-  // activation kernel at the start of every call; nothing else in the
-  // scratch has to start at a known value.
-  return w4a8_linear(x, M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
+  // activation kernel at the start of every call (the two-kernel path, also
+  // for one token); nothing else in the scratch has to start at a known value.
+  w4a8_status st = w4a8_linear_prepare(x, M, K, N, scratch, kStaticScratchBytes, stream);
+  if (st != W4A8_OK) return st;
+  return w4a8_linear_run(M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
 }
 
 w4a8_status w4a8_get_device_error(void* stream) {
