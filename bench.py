@@ -238,6 +238,144 @@ def run_reference(args) -> None:
 
 # ----------------------------------------------------------------------- GPU side
 
+C3_BLOCKS = 62
+C3_SHAPES = (("qkv", 5120, 10240), ("out", 5120, 5120), ("gate", 5120, 17408), ("up", 5120, 17408),
+             ("down", 17408, 5120))
+
+
+def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
+    """Down-projection shape K=17408, N=5120 at several token counts, 8 weight
+    copies cycled: M <= 16 runs the decode kernel, larger M the GEMM; the
+    per-call time shows where the GEMM takes over."""
+    k, n = 17408, 5120
+    copies = []
+    for c in range(COPIES):
+        q = synth.quantized_format_device(n, k, seed=2000 * (rank + 1) + c, device=dev)
+        copies.append(B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"]))
+        del q
+    wbytes = weight_bytes(n, k)
+    out = {}
+    for m in (1, 4, 16, 32, 64):
+        g = torch.Generator(device=dev)
+        g.manual_seed(300 + m)
+        x = torch.randn((m, k), generator=g, device=dev).to(torch.bfloat16)
+        ws = B.linear_workspace(m, k, n, dev)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        st = steps if m <= 16 else max(8, steps // 8)
+
+        def step(i):
+            B.linear(x, copies[i % COPIES], n, workspace=ws, out=y)
+
+        for i in range(warmup):
+            step(i)
+        replay = graph_loop(step, st, stream)
+        replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / st
+        out[f"M={m}"] = {"us_per_call": us, "weight_GBs": wbytes / us / 1e3,
+                         "us_per_token": us / m, "path": "decode" if m <= 16 else "tensor-core GEMM"}
+        del replay
+    del copies
+    torch.cuda.empty_cache()
+    return {"workload": f"K={k} N={n}, 8 weight copies cycled, one w4a8_linear per call", "by_m": out}
+
+
+def measure_c3(B, synth, torch, dev, rank, stream, steps, warmup):
+    """Decode step of a 62-block stack of projections, M=1, all weights
+    distinct and resident.  Per block the projections run as a chain:
+    h -> qkv (10240) -> out (its first 5120) -> gate and up (17408 each) ->
+    down (from up) -> next h; every call is one w4a8_linear."""
+    layers = []
+    total = 0
+    for b in range(C3_BLOCKS):
+        blk = []
+        for j, (name, k, n) in enumerate(C3_SHAPES):
+            q = synth.quantized_format_device(n, k, seed=100000 * (rank + 1) + 10 * b + j, device=dev)
+            blk.append((B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"]), k, n))
+            del q
+            total += weight_bytes(n, k)
+        layers.append(blk)
+    resident = sum(pk.numel() for blk in layers for pk, _, _ in blk)
+    ws = B.linear_workspace(1, 17408, 17408, dev)
+    need = max(B.linear_workspace_bytes(1, k, n) for _, k, n in C3_SHAPES)
+    assert ws.numel() >= need
+    g = torch.Generator(device=dev)
+    g.manual_seed(7 + rank)
+    h0 = torch.randn((1, 5120), generator=g, device=dev).to(torch.bfloat16)
+    bufs = {n: torch.empty((1, n), dtype=torch.bfloat16, device=dev) for n in (5120, 10240, 17408)}
+    qkv_o, out_o = torch.empty((1, 10240), dtype=torch.bfloat16, device=dev), bufs[5120]
+    gate_o, up_o = torch.empty((1, 17408), dtype=torch.bfloat16, device=dev), bufs[17408]
+    h = torch.empty((1, 5120), dtype=torch.bfloat16, device=dev)
+
+    def step(_i):
+        x = h0
+        for blk in layers:
+            (wq, _, _), (wo, _, _), (wg, _, _), (wu, _, _), (wd, _, _) = blk
+            B.linear(x, wq, 10240, workspace=ws, out=qkv_o)
+            B.linear(qkv_o[:, :5120], wo, 5120, workspace=ws, out=out_o)
+            B.linear(out_o, wg, 17408, workspace=ws, out=gate_o)
+            B.linear(out_o, wu, 17408, workspace=ws, out=up_o)
+            B.linear(up_o, wd, 5120, workspace=ws, out=h)
+            x = h
+
+    for i in range(warmup):
+        step(i)
+    replay = graph_loop(step, steps, stream, chunk=4)
+    replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    finite = bool(torch.isfinite(h.float()).all().item())
+    del replay, layers
+    torch.cuda.empty_cache()
+    return {"workload": f"{C3_BLOCKS} blocks x (qkv 5120->10240, out 5120->5120, gate/up 5120->17408, "
+                        "down 17408->5120), M=1, chained",
+            "ms_per_step": ms, "weight_GBs": total / (ms * 1e-3) / 1e9, "weight_bytes_per_step": total,
+            "resident_bytes": resident, "kernels_per_step": C3_BLOCKS * len(C3_SHAPES), "steps": steps,
+            "output_finite": finite}
+
+
+def measure_c4b(B, synth, torch, dev, rank, stream, steps, warmup):
+    """Second prefill shape: M=8192, K=17408, N=5120 (one w4a8_linear per step)."""
+    m, k, n = 8192, 17408, 5120
+    q = synth.quantized_format_device(n, k, seed=88 + rank, device=dev)
+    pk = B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"])
+    del q
+    g = torch.Generator(device=dev)
+    g.manual_seed(9 + rank)
+    x = torch.randn((m, k), generator=g, device=dev).to(torch.bfloat16)
+    ws = B.linear_workspace(m, k, n, dev)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+
+    def step(_i):
+        B.linear(x, pk, n, workspace=ws, out=y)
+
+    for i in range(warmup):
+        step(i)
+    replay = graph_loop(step, steps, stream)
+    replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del replay, pk, x, ws, y
+    torch.cuda.empty_cache()
+    return {"workload": f"prefill GEMM M={m} K={k} N={n}", "ms_per_step": ms,
+            "TOPS": 2.0 * m * n * k / (ms * 1e-3) / 1e12}
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -246,6 +384,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--prefill-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the C2/C3/second-prefill lines")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -404,6 +543,13 @@ def main() -> None:
         gemm_ms = max_over_ranks(q0.elapsed_time(q1)) / args.prefill_steps
     del replay_pre, replay_gemm
     pre_clocks = psampler.summary()
+
+    # ---------------- the other configurations: C2 token sweep, C3 decode step, C4 second shape
+    extra = {}
+    if not args.no_extra:
+        extra["c2_down_proj"] = measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup)
+        extra["c3_decode_step"] = measure_c3(B, synth, torch, dev, rank, stream, 20, 3)
+        extra["c4_prefill_8192"] = measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3)
     err = B.get_device_error()
 
     if world > 1:
@@ -465,6 +611,7 @@ def main() -> None:
                 "how": "per-step host loop through the Python binding: pinned x copied in, w4a8_linear, y copied out"},
         "clocks": dec_clocks,
         "gpu_launches": args.steps,
+        "other_configs": extra,
         "device_error": err,
     }
     if not args.no_cpu_baseline:

@@ -138,9 +138,9 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   y          output [M, N] bf16 bit patterns (uint16), row-major.
  *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
  * M <= 16 runs the decode kernel (a weight-streaming GEMV); larger M runs
- * the tensor-core GEMM.  For one token with K <= 15872 a single kernel
- * rotates, quantises and applies the layer (every CTA quantises the token
- * itself, with the activation kernel's arithmetic); otherwise the call is
+ * the tensor-core GEMM.  For one token a single kernel rotates, quantises
+ * and applies the layer (every CTA quantises the token itself, with the
+ * activation kernel's arithmetic); otherwise the call is
  * w4a8_linear_prepare followed by w4a8_linear_run.  Two calls sharing one
  * workspace must be ordered on the GPU (same stream, or synchronised).
  * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA.

@@ -272,12 +272,12 @@ def test_prepare_once_run_several_layers(lib, m):
         check_linear(y_run.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
 
 
-@pytest.mark.parametrize("k", [5120, 15872, 16128])
+@pytest.mark.parametrize("k", [5120, 15872, 16128, 17408, 32768])
 def test_one_token_single_kernel_equals_two_kernel_path(lib, k):
-    """For one token and K <= 15872, w4a8_linear is one kernel that rotates and
-    quantises the token itself; it must give the same bits as the activation
-    kernel followed by the decode kernel (K = 16128 takes that path anyway),
-    and match the oracle."""
+    """For one token, w4a8_linear is one kernel that rotates and quantises the
+    token itself (K > ~16K: the blocks that do not fit in shared memory are
+    rotated a second time); it must give the same bits as the activation
+    kernel followed by the decode kernel, and match the oracle."""
     n = 592
     c = O.convert_weight(synth.weights(n, k, synth.rng_for(70, k, "weight")), sample_cap=2**16)
     packed = pack(lib, c)

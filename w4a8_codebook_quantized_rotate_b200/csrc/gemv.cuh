@@ -71,10 +71,7 @@ __host__ __device__ inline size_t dec_smem_bytes(int m, int k, bool single) {
          kDecSchRows * 4 + 64 + 128 + 64;
 }
 
-// Largest K of the kernel that rotates and quantises its token itself: the
-// fp32 rotated row is staged below the 64 KiB-aligned table, in the first
-// 64 KiB of the CTA's shared window less the 1 KiB the system reserves.
-constexpr int kDecFusedMaxK = 15872;
+
 
 // Ranges: warp w holds units [floor(w U / W), floor((w+1) U / W)); in 32-bit
 // arithmetic as w R + floor(w Rm / W) (w Rm < W^2 < 2^32).  w may be W.
@@ -334,8 +331,9 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 //
 // FUSED (one token): the kernel also does the activation step: every CTA
 // rotates the bf16 row and quantises it to int8 (the activation kernel's
-// arithmetic, so the codes and s_x are the same bits), staging the rotated
-// row in fp32 below the table.  One launch then makes the whole layer.
+// arithmetic, so the codes and s_x are the same bits).  The rotated row is
+// staged in fp32 below the table as far as it fits (about 63 of the
+// 256-blocks); blocks past that are rotated again when they are quantised.  One launch then makes the whole layer.
 template <int NB, int D, bool SINGLE, bool FUSED = false>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
   static_assert(!FUSED || SINGLE, "the fused activation step handles one token");
@@ -352,11 +350,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
   const uint32_t wbeg_s = sx_s + 64;                                      // warp range starts [17]
   const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
-  const uint32_t rot_s = (base + 15u) & ~15u;                             // FUSED: rotated row [K] fp32
-  if (FUSED && rot_s + uint32_t(p.K) * 4u > lut) {  // the launch does not leave room below the table
-    if (threadIdx.x == 0) record_error(p.err, kErrTimeout);
-    return;
-  }
+  const uint32_t rot_s = (base + 15u) & ~15u;                             // FUSED: rotated row, fp32
+  // FUSED: 256-blocks of the rotated row that fit below the table
+  const int fit_blocks = min(p.K / kRotBlock, int((lut - rot_s) / (kRotBlock * 4u)));
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int cta_w0 = blockIdx.x * kDecWarps;
   const int w = cta_w0 + wl;
@@ -411,16 +407,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   int cx = first_c;  // chunk of the next x fragment to load (more than one token)
   if constexpr (FUSED) {
     // Rotate the row (warp per 256-block) and find its absmax.
+    const int nblk = p.K / kRotBlock;
     float amax = 0.f;
-    for (int b = wl; b < p.K / kRotBlock; b += kDecWarps) {
+    for (int b = wl; b < nblk; b += kDecWarps) {
       float v[8];
       rotate_block_lane(p.x, b, lane, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const uint32_t dst = rot_s + uint32_t(b * kRotBlock + lane * 8) * 4u;
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]), "f"(v[6]),
-                   "f"(v[7]));
+      if (b < fit_blocks) {
+        const uint32_t dst = rot_s + uint32_t(b * kRotBlock + lane * 8) * 4u;
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                     "f"(v[3]));
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+                     "f"(v[7]));
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -435,18 +435,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     const float s = quant_scale(amax);
     if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s), "f"(s));
     // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
-    // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4.
-    for (int k0 = threadIdx.x * 8; k0 < p.K; k0 += kDecThreads * 8) {
-      float v[8];
-      const uint32_t src = rot_s + uint32_t(k0) * 4u;
-      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(src));
-      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(src + 16u));
+    // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4; a run
+    // of 8 values from k0 (a multiple of 8) covers t = 0..3.
+    auto put_codes = [&](int k0, const float (&v)[8]) {
       const uint32_t dst = xs + uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const __half2 h = __floats2half2_rn(quant_code(v[2 * t], s), quant_code(v[2 * t + 1], s));
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + uint32_t(t) * 32u), "r"(*reinterpret_cast<const uint32_t*>(&h)));
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + uint32_t(t) * 32u),
+                     "r"(*reinterpret_cast<const uint32_t*>(&h)));
       }
+    };
+    for (int k0 = threadIdx.x * 8; k0 < fit_blocks * kRotBlock; k0 += kDecThreads * 8) {
+      float v[8];
+      const uint32_t src = rot_s + uint32_t(k0) * 4u;
+      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(src));
+      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(src + 16u));
+      put_codes(k0, v);
+    }
+    for (int b = fit_blocks + wl; b < nblk; b += kDecWarps) {  // blocks that did not fit: rotate again
+      float v[8];
+      rotate_block_lane(p.x, b, lane, v);
+      put_codes(b * kRotBlock + lane * 8, v);
     }
   } else {
     if (threadIdx.x < p.M)

@@ -76,8 +76,7 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Frag>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepthSingle, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
-          allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kDecFusedMaxK, true)) !=
-              cudaSuccess ||
+          allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
           allow_smem(decode_kernel<2, kDecDepth2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
@@ -234,9 +233,9 @@ static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* wo
   return device_state(d);
 }
 
-// Decode launch (M <= 16).  With x given (one token, K <= kDecFusedMaxK) the
-// kernel also rotates and quantises the token; otherwise it reads what
-// w4a8_linear_prepare left in the workspace.
+// Decode launch (M <= 16).  With x given (one token) the kernel also rotates
+// and quantises the token; otherwise it reads what w4a8_linear_prepare left
+// in the workspace.
 static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, int64_t M, int64_t K, int64_t N,
                                  const uint8_t* pk, uint16_t* y, uint8_t* ws, cudaStream_t s, const uint16_t* x) {
   const PackedLayout L = packed_layout(N, K);
@@ -347,7 +346,7 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* pac
                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !packed || !y || !workspace) return W4A8_ERR_NULL;
   if (!aligned16(packed) || !aligned16(y)) return W4A8_ERR_ALIGN;
-  if (M == 1 && K <= kDecFusedMaxK) {  // one token: a single kernel makes the layer
+  if (M == 1) {  // one token: a single kernel makes the layer
     if (!aligned16(x)) return W4A8_ERR_ALIGN;
     LinearPlan plan;
     DeviceState* d = nullptr;
