@@ -376,6 +376,43 @@ def measure_c4b(B, synth, torch, dev, rank, stream, steps, warmup):
             "TOPS": 2.0 * m * n * k / (ms * 1e-3) / 1e12}
 
 
+def measure_converter(B, torch, dev, rank, stream, reps=5):
+    """GPU weight converter on the C1 layer's shape: fp32 W [17408, 5120] ->
+    the four stored tensors.  'assign' = given codebook (rotation, scales,
+    indices); 'fit' = Lloyd-Max on a 2^22-value seeded sample first."""
+    import numpy as np
+    n, k = N_DEC, K_DEC
+    g = torch.Generator(device=dev)
+    g.manual_seed(11 + rank)
+    w = torch.randn((n, k), generator=g, device=dev) * 0.02
+    first = B.convert_weight_sampled(w, sample_cap=2 ** 22, seed=42)
+    pos = B.fit_sample_positions(first["s_rel"].cpu().numpy(), first["s_ch"].cpu().numpy(), 2 ** 22, 42)
+    pos_d = None if pos is None else torch.from_numpy(np.ascontiguousarray(pos)).to(dev)
+    cb = first["cb"].clone()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    assign_ms = timed(lambda: B.convert_weight(w, codebook=cb))
+    fit_ms = timed(lambda: B.convert_weight(w, sample_pos=pos_d))
+    rounds = int(first["fit_rounds"].item())
+    wb = n * k * 4
+    del w, first, pos_d
+    torch.cuda.empty_cache()
+    return {"workload": f"fp32 W [{n}, {k}] -> packed indices, e4m3 group scales, fp32 row scales, codebook",
+            "assign_ms": assign_ms, "assign_W_GBs": wb / (assign_ms * 1e-3) / 1e9,
+            "fit_ms": fit_ms, "fit_rounds": rounds, "fit_sample": 2 ** 22,
+            "note": "fp64 rotation and decisions (bit-exact with the oracle given the codebook)"}
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -550,6 +587,7 @@ def main() -> None:
         extra["c2_down_proj"] = measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup)
         extra["c3_decode_step"] = measure_c3(B, synth, torch, dev, rank, stream, 20, 3)
         extra["c4_prefill_8192"] = measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3)
+        extra["weight_converter"] = measure_converter(B, torch, dev, rank, stream)
     err = B.get_device_error()
 
     if world > 1:

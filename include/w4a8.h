@@ -55,7 +55,8 @@ typedef enum w4a8_status {
   W4A8_ERR_WORKSPACE = 4,  /* a buffer is smaller than the size function says */
   W4A8_ERR_CUDA = 5,       /* a CUDA call failed (launch or device query) */
   W4A8_ERR_TIMEOUT = 6,    /* a bounded device wait gave up (see get_device_error) */
-  W4A8_ERR_ARCH = 7        /* the current device is not sm_100 */
+  W4A8_ERR_ARCH = 7,       /* the current device is not sm_100 */
+  W4A8_ERR_INPUT = 8       /* a device-side input check failed (see get_device_error) */
 } w4a8_status;
 
 /*
@@ -203,10 +204,55 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K,
                                       void* stream);
 
 /*
+ * Weight converter on the GPU: fp32 W [N, K] -> the four stored tensors
+ * (ConvRot card, "Format": rotate by the group-256 Hadamard, a per-row scale
+ * and a per-16 e4m3 scale, 16-level Lloyd-Max codebook, two indices per
+ * byte; "Reproducing": the codebook fit samples the values with a fixed
+ * seed).  Per row, in fp64:
+ *   R = W rotated (each 256-block times H_256 / 16)
+ *   s_channel[n]  = fp32(max_k |R[n,k]|)
+ *   s_rel[n, g]   = e4m3 (round half to even, saturating) of
+ *                   max_{k in g} |R[n,k]| / s_channel[n]   (0 if s_channel is 0)
+ *   v[n, k]       = R[n,k] / (s_rel[n, g] * s_channel[n])  (0 where that is 0)
+ *   idx[n, k]     = the number of midpoints between consecutive codebook
+ *                   levels that are strictly below v (a value on a midpoint
+ *                   takes the lower level)
+ * With `codebook_in` given (16 fp32 levels, strictly ascending) those levels
+ * are used.  With `codebook_in` NULL the levels are fitted first (Lloyd-Max):
+ * the fit uses v at `sample_pos` (n_sample flat positions n*K + k, each a
+ * position whose group scale and row scale are non-zero; the caller draws
+ * them), or every such value when `sample_pos` is NULL; it starts at the
+ * sample's (i + 1/2)/16 quantiles (linear interpolation between order
+ * statistics) and alternates boundaries = level midpoints (a value on a
+ * midpoint belongs to the lower cell) and level = mean of its cell (an empty
+ * cell keeps its level) until no level moves by `tol` or after `max_iter`
+ * rounds.  Cell sums are exact (128-bit fixed point).
+ *   w            [N, K] fp32, row-major, 16-byte aligned.
+ *   idx_packed   out [N, K/2] uint8 (low nibble = even k).
+ *   s_rel        out [N, K/16] uint8 e4m3fn codes.
+ *   s_channel    out [N] fp32.
+ *   codebook_out out [16] fp32 (the fitted levels, or a copy of codebook_in).
+ *   fit_rounds   out, device int32 (rounds the fit took; 0 when given), or NULL.
+ *   workspace    w4a8_convert_workspace_bytes(N, K, n_sample) bytes (only
+ *                the fit uses it; n_sample <= 0 sizes it for every value).
+ * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA; an out-of-range sample
+ * position or an empty sample is reported by w4a8_get_device_error as
+ * W4A8_ERR_INPUT.
+ */
+size_t w4a8_convert_workspace_bytes(int64_t N, int64_t K, int64_t n_sample);
+w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const float* codebook_in,
+                                const int64_t* sample_pos, int64_t n_sample, int32_t max_iter,
+                                double tol, uint8_t* idx_packed, uint8_t* s_rel,
+                                float* s_channel, float* codebook_out, int32_t* fit_rounds,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then report and clear the device-side error word of
  * the current device: W4A8_ERR_TIMEOUT if a bounded wait inside a kernel
  * gave up since the last call (the affected outputs are then undefined),
- * W4A8_ERR_CUDA if the synchronisation itself failed, else W4A8_OK.
+ * W4A8_ERR_INPUT if a kernel found an input it cannot use (a converter
+ * sample position out of range, or an empty sample), W4A8_ERR_CUDA if the
+ * synchronisation itself failed, else W4A8_OK.
  */
 w4a8_status w4a8_get_device_error(void* stream);
 

@@ -27,6 +27,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
+        "w4a8_convert_weight", "w4a8_convert_workspace_bytes",
         "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_prepare",
         "w4a8_linear_run",
         "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
@@ -91,3 +92,18 @@ def test_status_strings(lib):
     for s in range(8):
         assert lib.w4a8_status_string(s)
     assert b"unknown" in lib.w4a8_status_string(99)
+
+
+def test_convert_workspace_sizes(lib):
+    assert lib.w4a8_convert_workspace_bytes(16, 256, 0) > 16 * 256 * 8
+    assert lib.w4a8_convert_workspace_bytes(16, 300, 0) == 0
+    assert lib.w4a8_convert_workspace_bytes(16, 256, 16 * 256 + 1) == 0   # more positions than values
+    small = lib.w4a8_convert_workspace_bytes(17408, 5120, 2 ** 22)
+    whole = lib.w4a8_convert_workspace_bytes(17408, 5120, 0)
+    assert 2 ** 22 * 24 < small < whole
+
+
+def test_convert_refuses_bad_arguments_without_a_gpu(lib):
+    # null pointers and shapes are checked before any device work
+    assert lib.w4a8_convert_weight(None, 16, 256, None, None, 0, 500, 1e-12, None, None, None, None, None,
+                                   None, 0, None) == 1

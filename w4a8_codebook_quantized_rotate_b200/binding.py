@@ -18,12 +18,14 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libw
 STATUS = {
     0: "ok", 1: "null pointer", 2: "bad shape", 3: "misaligned pointer",
     4: "buffer too small", 5: "CUDA error", 6: "device wait timed out", 7: "device is not sm_100",
+    8: "device-side input check failed",
 }
 
 EXPORTS = (
     "w4a8_packed_bytes", "w4a8_pack_layout", "w4a8_unpack_dequant", "w4a8_rotate_quant_act",
     "w4a8_linear_workspace_bytes", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
     "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_status_string",
+    "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
 )
 
 _lib = None
@@ -56,6 +58,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_linear_decode_static": (st, [vp, i64, i64, vp, i64, vp, vp]),
         "w4a8_get_device_error": (st, [vp]),
         "w4a8_status_string": (ctypes.c_char_p, [st]),
+        "w4a8_convert_workspace_bytes": (sz, [i64, i64, i64]),
+        "w4a8_convert_weight": (st, [vp, i64, i64, vp, vp, i64, ctypes.c_int32, ctypes.c_double,
+                                     vp, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -206,3 +211,69 @@ def linear_decode_static(x: torch.Tensor, packed: torch.Tensor, n: int, out: tor
 def get_device_error(stream=None) -> int:
     """Synchronise and return (and clear) the device error status (0 = ok)."""
     return int(load_library().w4a8_get_device_error(_stream(stream)))
+
+
+def convert_weight(w: torch.Tensor, codebook: torch.Tensor | None = None, sample_pos: torch.Tensor | None = None,
+                   max_iter: int = 500, tol: float = 1e-12, stream=None) -> dict:
+    """fp32 W [N, K] on the GPU -> the four stored tensors (``packed`` [N, K/2] uint8,
+    ``s_rel`` [N, K/16] uint8 e4m3 codes, ``s_ch`` [N] fp32, ``cb`` [16] fp32) and
+    ``fit_rounds``.  With ``codebook`` given its levels are used; otherwise they are
+    fitted on the values at ``sample_pos`` (int64 flat positions), or on every
+    value whose scales are non-zero when ``sample_pos`` is None."""
+    lib = load_library()
+    _cuda(w, torch.float32, "w")
+    n, k = w.shape
+    dev = w.device
+    packed = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+    s_rel = torch.empty((n, k // 16), dtype=torch.uint8, device=dev)
+    s_ch = torch.empty((n,), dtype=torch.float32, device=dev)
+    cb = torch.empty((16,), dtype=torch.float32, device=dev)
+    rounds = torch.zeros((1,), dtype=torch.int32, device=dev)
+    ws, ws_ptr, ws_bytes = None, None, 0
+    cb_ptr, pos_ptr, n_pos = None, None, 0
+    if codebook is not None:
+        _cuda(codebook, torch.float32, "codebook")
+        cb_ptr = codebook.data_ptr()
+    else:
+        if sample_pos is not None:
+            _cuda(sample_pos, torch.int64, "sample_pos")
+            pos_ptr, n_pos = sample_pos.data_ptr(), sample_pos.numel()
+        ws_bytes = lib.w4a8_convert_workspace_bytes(n, k, n_pos)
+        if ws_bytes == 0:
+            raise W4A8Error("w4a8_convert_workspace_bytes", 2)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        ws_ptr = ws.data_ptr()
+    _check("w4a8_convert_weight", lib.w4a8_convert_weight(
+        w.data_ptr(), n, k, cb_ptr, pos_ptr, n_pos, int(max_iter), float(tol), packed.data_ptr(),
+        s_rel.data_ptr(), s_ch.data_ptr(), cb.data_ptr(), rounds.data_ptr(), ws_ptr, ws_bytes, _stream(stream)))
+    return {"packed": packed, "s_rel": s_rel, "s_ch": s_ch, "cb": cb, "fit_rounds": rounds, "workspace": ws}
+
+
+def fit_sample_positions(s_rel: "np.ndarray", s_ch: "np.ndarray", cap: int, seed: int):
+    """Flat positions (n K + k) of a codebook-fit sample: the values whose group
+    and row scales are non-zero, in row-major order, form the pool; if it holds
+    more than ``cap`` values, ``cap`` of them are drawn without replacement by
+    numpy's PCG64 generator seeded with ``seed`` (Generator.choice over the pool
+    size); else None (fit on the whole pool)."""
+    import numpy as np
+    s_rel = np.asarray(s_rel, dtype=np.uint8)
+    live = ((s_rel & 0x7F) != 0) & (np.asarray(s_ch) > 0)[:, None]
+    groups = np.flatnonzero(live.ravel())
+    n_live = groups.size * 16
+    if n_live <= cap:
+        return None
+    p = np.random.Generator(np.random.PCG64(seed)).choice(n_live, size=cap, replace=False)
+    return groups[p // 16].astype(np.int64) * 16 + (p % 16)
+
+
+def convert_weight_sampled(w: torch.Tensor, sample_cap: int = 2 ** 22, seed: int = 42, max_iter: int = 500,
+                           tol: float = 1e-12, stream=None) -> dict:
+    """:func:`convert_weight` with the fit sample drawn as described in
+    :func:`fit_sample_positions` (the scales are computed first, with a
+    provisional codebook, to find the pool)."""
+    import numpy as np
+    provisional = torch.linspace(-1.0, 1.0, 16, dtype=torch.float32, device=w.device)
+    first = convert_weight(w, codebook=provisional, stream=stream)
+    pos = fit_sample_positions(first["s_rel"].cpu().numpy(), first["s_ch"].cpu().numpy(), sample_cap, seed)
+    sample = None if pos is None else torch.from_numpy(np.ascontiguousarray(pos)).to(w.device)
+    return convert_weight(w, sample_pos=sample, max_iter=max_iter, tol=tol, stream=stream)

@@ -51,6 +51,7 @@ constexpr int kMaxK = 32768;
 
 // Device-side error word values (bit flags).
 constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrInput = 2u;  // a device-side input check failed
 
 struct PackedLayout {
   int64_t N, K, tiles, pairs, chunks;

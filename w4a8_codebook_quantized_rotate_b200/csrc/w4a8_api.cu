@@ -7,6 +7,7 @@
 
 #include "act.cuh"
 #include "common.cuh"
+#include "convert.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
@@ -389,6 +390,100 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, c
   return w4a8_linear_run(M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
 }
 
+// ------------------------------------------------------------------ weight converter
+
+struct ConvertPlan {
+  int64_t n_cap, n_pad, scan_blocks;
+  size_t off_bits, off_samples, off_bsum, off_prefix, total;
+};
+
+static ConvertPlan convert_plan(int64_t N, int64_t K, int64_t n_sample) {
+  ConvertPlan c{};
+  c.n_cap = n_sample > 0 ? n_sample : N * K;
+  c.n_pad = int64_t(kBitonicTile);
+  while (c.n_pad < c.n_cap) c.n_pad <<= 1;
+  c.scan_blocks = (c.n_pad + kScanThreads * kScanItems - 1) / (kScanThreads * kScanItems);
+  c.off_bits = 256;  // [0, 8): sample counter
+  c.off_samples = round_up(c.off_bits + size_t((N * K + 63) / 64) * 8, 256);
+  c.off_bsum = round_up(c.off_samples + size_t(c.n_pad) * 8, 256);
+  c.off_prefix = round_up(c.off_bsum + size_t(c.scan_blocks + 1) * 16, 256);
+  c.total = round_up(c.off_prefix + size_t(c.n_pad + 1) * 16, 256);
+  return c;
+}
+
+size_t w4a8_convert_workspace_bytes(int64_t N, int64_t K, int64_t n_sample) {
+  if (!weight_shape_ok(N, K) || n_sample > N * K) return 0;
+  return convert_plan(N, K, n_sample).total;
+}
+
+w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const float* codebook_in,
+                                const int64_t* sample_pos, int64_t n_sample, int32_t max_iter, double tol,
+                                uint8_t* idx_packed, uint8_t* s_rel, float* s_channel, float* codebook_out,
+                                int32_t* fit_rounds, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!w || !idx_packed || !s_rel || !s_channel || !codebook_out) return W4A8_ERR_NULL;
+  if (!weight_shape_ok(N, K) || max_iter < 1 || !(tol >= 0.0)) return W4A8_ERR_SHAPE;
+  if (sample_pos && (n_sample < 1 || n_sample > N * K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(idx_packed)) return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CvtParams p{};
+  p.w = w;
+  p.idx = idx_packed;
+  p.s_rel = s_rel;
+  p.s_ch = s_channel;
+  p.N = N;
+  p.K = K;
+  const size_t smem = size_t(K / kGroup) * 8;
+  if (codebook_in) {
+    p.cb = codebook_in;
+    convert_row_kernel<0><<<unsigned(N), kCvtThreads, smem, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return W4A8_ERR_CUDA;
+    if (codebook_out != codebook_in &&
+        cudaMemcpyAsync(codebook_out, codebook_in, 16 * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return W4A8_ERR_CUDA;
+    if (fit_rounds && cudaMemsetAsync(fit_rounds, 0, sizeof(int32_t), s) != cudaSuccess) return W4A8_ERR_CUDA;
+    return W4A8_OK;
+  }
+  // fit the codebook first
+  if (!workspace) return W4A8_ERR_NULL;
+  if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+  const ConvertPlan c = convert_plan(N, K, sample_pos ? n_sample : 0);
+  if (workspace_bytes < c.total) return W4A8_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto* counter = reinterpret_cast<unsigned long long*>(ws);
+  auto* bits = reinterpret_cast<uint64_t*>(ws + c.off_bits);
+  auto* samples = reinterpret_cast<double*>(ws + c.off_samples);
+  auto* bsum = reinterpret_cast<__int128*>(ws + c.off_bsum);
+  auto* prefix = reinterpret_cast<__int128*>(ws + c.off_prefix);
+  const int fill_grid = int(d->sms) * 8;
+  if (cudaMemsetAsync(counter, 0, 8, s) != cudaSuccess) return W4A8_ERR_CUDA;
+  fill_u64_kernel<<<fill_grid, 256, 0, s>>>(reinterpret_cast<uint64_t*>(samples), c.n_pad,
+                                             0x7FF0000000000000ull);  // +inf: sorts past the sample
+  if (sample_pos) {
+    fill_u64_kernel<<<fill_grid, 256, 0, s>>>(bits, (N * K + 63) / 64, 0ull);
+    sample_bits_kernel<<<unsigned((n_sample + 255) / 256), 256, 0, s>>>(sample_pos, n_sample, bits, N * K, d->err);
+  }
+  p.sample_bits = sample_pos ? bits : nullptr;
+  p.samples = samples;
+  p.n_samples = counter;
+  convert_row_kernel<1><<<unsigned(N), kCvtThreads, smem, s>>>(p);
+  // sort (bitonic network; strides below the tile size run in shared memory)
+  const unsigned sort_grid = unsigned(c.n_pad / 256);
+  for (int64_t k = 2; k <= c.n_pad; k <<= 1) {
+    int64_t j = k >> 1;
+    for (; j >= kBitonicTile; j >>= 1) bitonic_step_kernel<<<sort_grid, 256, 0, s>>>(samples, c.n_pad, j, k);
+    bitonic_local_kernel<<<unsigned(c.n_pad / kBitonicTile), kBitonicTile / 2, 0, s>>>(samples, k, j);
+  }
+  scan_blocks_kernel<<<unsigned(c.scan_blocks), kScanThreads, 0, s>>>(samples, c.n_pad, bsum);
+  scan_offsets_kernel<<<1, 1, 0, s>>>(bsum, c.scan_blocks);
+  scan_final_kernel<<<unsigned(c.scan_blocks), kScanThreads, 0, s>>>(samples, c.n_pad, bsum, prefix);
+  lloyd_kernel<<<1, 32, 0, s>>>(samples, counter, prefix, max_iter, tol, codebook_out, fit_rounds, d->err);
+  p.cb = codebook_out;
+  convert_row_kernel<0><<<unsigned(N), kCvtThreads, smem, s>>>(p);
+  return launch_status();
+}
+
 w4a8_status w4a8_get_device_error(void* stream) {
   DeviceState* d = nullptr;
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
@@ -399,7 +494,8 @@ w4a8_status w4a8_get_device_error(void* stream) {
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
   }
-  return (v & kErrTimeout) ? W4A8_ERR_TIMEOUT : W4A8_OK;
+  if (v & kErrTimeout) return W4A8_ERR_TIMEOUT;
+  return (v & kErrInput) ? W4A8_ERR_INPUT : W4A8_OK;
 }
 
 const char* w4a8_status_string(w4a8_status status) {
@@ -412,6 +508,7 @@ const char* w4a8_status_string(w4a8_status status) {
     case W4A8_ERR_CUDA: return "a CUDA call failed";
     case W4A8_ERR_TIMEOUT: return "a bounded device wait gave up";
     case W4A8_ERR_ARCH: return "the current device is not sm_100";
+    case W4A8_ERR_INPUT: return "a device-side input check failed";
   }
   return "unknown status";
 }
