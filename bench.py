@@ -405,12 +405,26 @@ def measure_converter(B, torch, dev, rank, stream, reps=5):
     fit_ms = timed(lambda: B.convert_weight(w, sample_pos=pos_d))
     rounds = int(first["fit_rounds"].item())
     wb = n * k * 4
-    del w, first, pos_d
+    # fidelity check of the converted layer against its source (host-side sample draw included)
+    packed = B.pack_layout(first["packed"], first["s_rel"], first["s_ch"], first["cb"])
+    xg = torch.Generator(device=dev)
+    xg.manual_seed(12 + rank)
+    x = torch.randn((4, k), generator=xg, device=dev).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ver = B.verify_layer(w, packed, x)
+    torch.cuda.synchronize()
+    verify_ms = (time.perf_counter() - t0) * 1e3
+    del w, first, pos_d, packed
     torch.cuda.empty_cache()
     return {"workload": f"fp32 W [{n}, {k}] -> packed indices, e4m3 group scales, fp32 row scales, codebook",
             "assign_ms": assign_ms, "assign_W_GBs": wb / (assign_ms * 1e-3) / 1e9,
             "fit_ms": fit_ms, "fit_rounds": rounds, "fit_sample": 2 ** 22,
-            "note": "fp64 rotation and decisions (bit-exact with the oracle given the codebook)"}
+            "note": "fp64 rotation and decisions (bit-exact with the oracle given the codebook)",
+            "verify": {"fidelity": ver["fidelity"], "forward_error_4_tokens": ver["forward"],
+                       "wall_ms": verify_ms,
+                       "note": "stored = this conversion; fresh re-conversion with the seeded fit; "
+                               "wall time includes the host-side sample draw"}}
 
 
 def main() -> None:

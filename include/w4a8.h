@@ -247,6 +247,30 @@ w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const floa
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Fidelity checks of a stored layer (ConvRot card, "Verification": a stored
+ * layer's dequantised weights compared with a fresh quantisation of the same
+ * source tensor, expected ~0; "Accuracy": the quantised layer's output
+ * against the full-precision one, ~1 %).  The binding's verify_layer
+ * composes them with w4a8_convert_weight, w4a8_unpack_dequant and
+ * w4a8_linear.
+ *
+ * w4a8_compare: out[0] = sum_i (a[i] - ref[i])^2, out[1] = sum_i ref[i]^2,
+ *   out[2] = max_i |a[i] - ref[i]|, all in fp64 (device memory, 8-byte
+ *   aligned).  a is fp32 (a_is_bf16 = 0) or bf16 bit patterns (1); ref is
+ *   fp32; n values each.  The reduction order is fixed (same result on every
+ *   call and device).  workspace: w4a8_compare_workspace_bytes() bytes.
+ *   Errors: NULL, SHAPE, WORKSPACE, ALIGN, ARCH, CUDA.
+ * w4a8_dense_reference: y [M, N] fp32 = x [M, K] (bf16 bits) times W^T
+ *   (W [N, K] fp32, unquantised, original basis), each sum in fp64 then
+ *   rounded once.  Errors: NULL, SHAPE, ARCH, CUDA.
+ */
+size_t w4a8_compare_workspace_bytes(void);
+w4a8_status w4a8_compare(const void* a, int32_t a_is_bf16, const float* ref, int64_t n,
+                         double* out, void* workspace, size_t workspace_bytes, void* stream);
+w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const float* w,
+                                 int64_t N, float* y, void* stream);
+
+/*
  * Synchronise `stream`, then report and clear the device-side error word of
  * the current device: W4A8_ERR_TIMEOUT if a bounded wait inside a kernel
  * gave up since the last call (the affected outputs are then undefined),

@@ -26,6 +26,7 @@ EXPORTS = (
     "w4a8_linear_workspace_bytes", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
     "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_status_string",
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
+    "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
 )
 
 _lib = None
@@ -61,6 +62,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_convert_workspace_bytes": (sz, [i64, i64, i64]),
         "w4a8_convert_weight": (st, [vp, i64, i64, vp, vp, i64, ctypes.c_int32, ctypes.c_double,
                                      vp, vp, vp, vp, vp, vp, sz, vp]),
+        "w4a8_compare_workspace_bytes": (sz, []),
+        "w4a8_compare": (st, [vp, ctypes.c_int32, vp, i64, vp, vp, sz, vp]),
+        "w4a8_dense_reference": (st, [vp, i64, i64, vp, i64, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -277,3 +281,56 @@ def convert_weight_sampled(w: torch.Tensor, sample_cap: int = 2 ** 22, seed: int
     pos = fit_sample_positions(first["s_rel"].cpu().numpy(), first["s_ch"].cpu().numpy(), sample_cap, seed)
     sample = None if pos is None else torch.from_numpy(np.ascontiguousarray(pos)).to(w.device)
     return convert_weight(w, sample_pos=sample, max_iter=max_iter, tol=tol, stream=stream)
+
+
+def compare(a: torch.Tensor, ref: torch.Tensor, stream=None) -> torch.Tensor:
+    """fp64 device tensor [sum (a - ref)^2, sum ref^2, max |a - ref|]; a fp32 or bf16, ref fp32."""
+    lib = load_library()
+    if a.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("a must be fp32 or bf16")
+    _cuda(a, a.dtype, "a")
+    _cuda(ref, torch.float32, "ref")
+    if a.numel() != ref.numel():
+        raise ValueError("a and ref differ in size")
+    out = torch.empty(3, dtype=torch.float64, device=a.device)
+    ws = torch.empty(lib.w4a8_compare_workspace_bytes(), dtype=torch.uint8, device=a.device)
+    _check("w4a8_compare", lib.w4a8_compare(a.data_ptr(), int(a.dtype == torch.bfloat16), ref.data_ptr(),
+                                            a.numel(), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+def dense_reference(x: torch.Tensor, w: torch.Tensor, stream=None) -> torch.Tensor:
+    """Unquantised layer: fp32 y [M, N] = bf16 x [M, K] times fp32 W [N, K]^T (fp64 sums)."""
+    lib = load_library()
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w, torch.float32, "w")
+    m, k = x.shape
+    n = w.shape[0]
+    if w.shape[1] != k:
+        raise ValueError("x and w disagree on K")
+    y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _check("w4a8_dense_reference", lib.w4a8_dense_reference(x.data_ptr(), m, k, w.data_ptr(), n, y.data_ptr(),
+                                                            _stream(stream)))
+    return y
+
+
+def verify_layer(w: torch.Tensor, packed: torch.Tensor, x: torch.Tensor, sample_cap: int = 2 ** 22,
+                 seed: int = 42, stream=None) -> dict:
+    """Fidelity of a stored layer (``packed``, from :func:`pack_layout`) to its fp32
+    source ``w`` [N, K]: ``fidelity`` = relative L2 distance between the stored
+    layer's dequantised weights and those of a fresh conversion of ``w`` (seeded
+    fit), ~0 for a faithful file; ``forward`` = relative L2 error of the stored
+    layer's output on the probe activations ``x`` [M, K] (bf16) against the
+    unquantised x W^T."""
+    n, k = w.shape
+    fresh = convert_weight_sampled(w, sample_cap=sample_cap, seed=seed, stream=stream)
+    packed_fresh = pack_layout(fresh["packed"], fresh["s_rel"], fresh["s_ch"], fresh["cb"], stream=stream)
+    w_file = unpack_dequant(packed, n, k, stream=stream)
+    w_fresh = unpack_dequant(packed_fresh, n, k, stream=stream)
+    c1 = compare(w_file, w_fresh, stream=stream).cpu()
+    y_q = linear(x, packed, n, stream=stream)
+    y_ref = dense_reference(x, w, stream=stream)
+    c2 = compare(y_q, y_ref, stream=stream).cpu()
+    rel = lambda c: float((c[0] / c[1]).sqrt()) if c[1] > 0 else float(c[0] > 0)
+    return {"fidelity": rel(c1), "fidelity_max_abs": float(c1[2]), "forward": rel(c2),
+            "forward_max_abs": float(c2[2]), "fit_rounds": int(fresh["fit_rounds"].item())}

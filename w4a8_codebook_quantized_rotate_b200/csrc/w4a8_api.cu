@@ -11,6 +11,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
+#include "verify.cuh"
 
 namespace w4a8 {
 
@@ -481,6 +482,37 @@ w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const floa
   lloyd_kernel<<<1, 32, 0, s>>>(samples, counter, prefix, max_iter, tol, codebook_out, fit_rounds, d->err);
   p.cb = codebook_out;
   convert_row_kernel<0><<<unsigned(N), kCvtThreads, smem, s>>>(p);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ fidelity checks
+
+size_t w4a8_compare_workspace_bytes(void) { return size_t(kCmpBlocks) * 3 * sizeof(double); }
+
+w4a8_status w4a8_compare(const void* a, int32_t a_is_bf16, const float* ref, int64_t n, double* out,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!a || !ref || !out || !workspace) return W4A8_ERR_NULL;
+  if (n < 1) return W4A8_ERR_SHAPE;
+  if (workspace_bytes < w4a8_compare_workspace_bytes()) return W4A8_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) || (reinterpret_cast<uintptr_t>(workspace) & 7u)) return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(workspace);
+  if (a_is_bf16) compare_kernel<true><<<kCmpBlocks, kCmpThreads, 0, s>>>(a, ref, n, part);
+  else compare_kernel<false><<<kCmpBlocks, kCmpThreads, 0, s>>>(a, ref, n, part);
+  compare_final_kernel<<<1, 32, 0, s>>>(part, out);
+  return launch_status();
+}
+
+w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const float* w, int64_t N, float* y,
+                                 void* stream) {
+  if (!x || !w || !y) return W4A8_ERR_NULL;
+  if (M < 1 || M > (int64_t(1) << 24) || K < 1 || N < 1 || N > (int64_t(1) << 30)) return W4A8_ERR_SHAPE;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  dense_reference_kernel<<<unsigned((N + kRefWarps - 1) / kRefWarps), kRefWarps * 32, 0,
+                           static_cast<cudaStream_t>(stream)>>>(x, M, K, w, N, y);
   return launch_status();
 }
 
