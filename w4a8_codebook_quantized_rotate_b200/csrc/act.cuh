@@ -161,4 +161,81 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
   }
 }
 
+// The decode operand for a few tokens, one token per thread-block cluster:
+// CTA c of the cluster rotates 256-blocks [16 c, 16 c + 16) (a warp each,
+// the values stay in registers), the CTAs exchange their absmax through
+// distributed shared memory, and each quantises its own blocks.  Same
+// arithmetic as rotate_quant_kernel (rotate_block_lane, quant_scale,
+// quant_code): the same codes and s_x.  Splitting the token over up to 8
+// SMs cuts the latency of the step before a decode GEMV.
+constexpr int kActClusterBlocks = 16;  // 256-blocks per CTA (one per warp)
+constexpr int kActClusterThreads = kActClusterBlocks * 32;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Reads a float at a shared address of CTA `rank` of this cluster.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_kernel(
+    const uint16_t* __restrict__ x, int M, int K, __half2* __restrict__ out, float* __restrict__ s_x, int nb,
+    unsigned* __restrict__ zero_words, int zero_count) {
+  __shared__ float warp_max[kActClusterBlocks];
+  __shared__ float cta_max;
+  // The previous kernel may still read the workspace: wait before writing.
+  pdl_wait();
+  pdl_launch_dependents();
+  const int m = blockIdx.y;
+  const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (zero_words && m == 0 && rank == 0) {
+    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_words[i] = 0u;
+  }
+  const int b = int(rank) * kActClusterBlocks + warp;
+  const bool mine = b < K / kRotBlock;
+  float v[8];
+  float amax = 0.f;
+  if (mine) {
+    rotate_block_lane(x + int64_t(m) * K, b, lane, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = warp_max[0];
+    for (int i = 1; i < kActClusterBlocks; ++i) a = fmaxf(a, warp_max[i]);
+    cta_max = a;
+  }
+  cluster_sync_all();  // every CTA's maximum is written and visible cluster-wide
+  float tmax = 0.f;
+  for (uint32_t r = 0; r < ncta; ++r) tmax = fmaxf(tmax, ld_cluster_f32(smem_u32(&cta_max), r));
+  const float s = quant_scale(tmax);
+  if (rank == 0 && threadIdx.x == 0) s_x[m] = s;
+  if (mine) {
+    const int k0 = b * kRotBlock + lane * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[frag_half2_index(m, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], s), quant_code(v[2 * i + 1], s));
+  }
+  cluster_sync_all();  // no CTA leaves while another may still read its cta_max
+}
+
 }  // namespace w4a8

@@ -160,6 +160,27 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// launch_pdl with a 1-D thread-block cluster of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, unsigned cluster_x, size_t smem,
+                               cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 }  // namespace
 }  // namespace w4a8
 
@@ -288,9 +309,11 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* s_x = reinterpret_cast<float*>(ws + plan.off_sx);
   if (plan.decode) {
-    if (launch_pdl(rotate_quant_kernel<kActF16Frag>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
-                   int(M), int(K), (void*)(ws + plan.off_xq), s_x, plan.nb,
-                   reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P) != cudaSuccess)
+    // one cluster of up to 8 CTAs per token (16 blocks of 256 per CTA)
+    const unsigned cl = unsigned((K / kRotBlock + kActClusterBlocks - 1) / kActClusterBlocks);
+    if (launch_pdl_cluster(rotate_quant_frag_cluster_kernel, dim3(cl, unsigned(M)), dim3(kActClusterThreads), cl, 0,
+                           s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x, plan.nb,
+                           reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P) != cudaSuccess)
       return W4A8_ERR_CUDA;
   } else {
     if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
