@@ -245,8 +245,8 @@ C3_SHAPES = (("qkv", 5120, 10240), ("out", 5120, 5120), ("gate", 5120, 17408), (
 
 def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
     """Down-projection shape K=17408, N=5120 at several token counts, 8 weight
-    copies cycled: M <= 16 runs the decode kernel, larger M the GEMM; the
-    per-call time shows where the GEMM takes over."""
+    copies cycled: M <= 64 runs the decode kernel (one launch per 16 tokens),
+    larger M the GEMM; the per-call time shows where the GEMM takes over."""
     k, n = 17408, 5120
     copies = []
     for c in range(COPIES):
@@ -255,7 +255,7 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
         del q
     wbytes = weight_bytes(n, k)
     out = {}
-    for m in (1, 4, 16, 32, 64):
+    for m in (1, 4, 16, 32, 64, 128):
         g = torch.Generator(device=dev)
         g.manual_seed(300 + m)
         x = torch.randn((m, k), generator=g, device=dev).to(torch.bfloat16)
@@ -278,7 +278,8 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / st
         out[f"M={m}"] = {"us_per_call": us, "weight_GBs": wbytes / us / 1e3,
-                         "us_per_token": us / m, "path": "decode" if m <= 16 else "tensor-core GEMM"}
+                         "us_per_token": us / m,
+                         "path": "decode" if m <= 16 else "decode, slices of 16" if m <= 64 else "tensor-core GEMM"}
         del replay
     del copies
     torch.cuda.empty_cache()

@@ -138,8 +138,8 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   packed     a buffer filled by w4a8_pack_layout for the same (N, K).
  *   y          output [M, N] bf16 bit patterns (uint16), row-major.
  *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
- * M <= 16 runs the decode kernel (a weight-streaming GEMV); larger M runs
- * the tensor-core GEMM.  For one token a single kernel rotates, quantises
+ * M <= 64 runs the decode kernel (a weight-streaming GEMV, one launch per
+ * slice of up to 16 tokens); larger M runs the tensor-core GEMM.  For one token a single kernel rotates, quantises
  * and applies the layer (every CTA quantises the token itself, with the
  * activation kernel's arithmetic); otherwise the call is
  * w4a8_linear_prepare followed by w4a8_linear_run.  Two calls sharing one

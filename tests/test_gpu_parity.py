@@ -151,7 +151,21 @@ def test_linear_decode_matches_oracle(lib, layer592, m):
     check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
 
 
-@pytest.mark.parametrize("m", [17, 64, 255, 256, 300])
+@pytest.mark.parametrize("m", [17, 24, 33, 47, 64])
+def test_linear_sliced_decode_matches_oracle(lib, layer592, m):
+    """17..64 tokens run the decode kernel once per slice of 16 tokens (the
+    last slice ragged); prepare-then-run gives the same bits as the one call."""
+    c, packed, wmax = layer592
+    bits, x, _ = synth.activations(m, 768, synth.rng_for(12, m, "act"), 8)
+    y = run_linear(lib, bits, packed, 592)
+    check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+    ws = lib.linear_workspace(m, 768, 592, "cuda")
+    lib.linear_prepare(bf16(bits), 592, ws)
+    y2 = lib.linear_run(m, 768, packed, 592, ws).float().cpu().numpy()
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))
+
+
+@pytest.mark.parametrize("m", [65, 255, 256, 300])
 def test_linear_prefill_matches_oracle(lib, layer592, m):
     c, packed, wmax = layer592
     bits, x, _ = synth.activations(m, 768, synth.rng_for(5, m, "act"), 8)

@@ -22,7 +22,6 @@ namespace w4a8 {
 enum ActOut : int {
   kActI8Row = 0,    // int8 [M, K] row-major (the C ABI's rotate-quant call)
   kActF16Row = 1,   // fp16 [M, K] row-major, the tensor-core GEMM's operand
-  kActF16Frag = 2,  // fp16 in mma.sync B-fragment order, the decode kernel's operand
 };
 
 constexpr int kActMaxThreads = 1024;
@@ -91,9 +90,7 @@ __device__ __forceinline__ float quant_code(float v, float s) {
 
 template <int OUT>
 __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
-                                                                  void* __restrict__ out, float* __restrict__ s_x,
-                                                                  int nb, unsigned* __restrict__ zero_words,
-                                                                  int zero_count) {
+                                                                  void* __restrict__ out, float* __restrict__ s_x) {
   extern __shared__ float xr[];  // [K] rotated row
   __shared__ float warp_max[kActMaxThreads / 32];
   const int nwarps = blockDim.x >> 5;
@@ -104,9 +101,6 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
   pdl_launch_dependents();
   const int m = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (zero_words && m == 0) {
-    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_words[i] = 0u;
-  }
   const int nblocks = K / kRotBlock;
   float amax = 0.f;
   for (int b = warp; b < nblocks; b += nwarps) {
@@ -145,18 +139,12 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
         hi |= (uint32_t(int(q[i + 4])) & 0xFFu) << (8 * i);
       }
       *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + int64_t(m) * K + k0) = make_uint2(lo, hi);
-    } else if constexpr (OUT == kActF16Row) {
+    } else {
       __half2 h[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
       *reinterpret_cast<uint4*>(static_cast<__half*>(out) + int64_t(m) * K + k0) =
           *reinterpret_cast<uint4*>(h);
-    } else {
-      __half2* o = static_cast<__half2*>(out);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        o[frag_half2_index(m, k0 + 2 * i, nb)] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
-      }
     }
   }
 }
@@ -193,9 +181,12 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t ra
   return v;
 }
 
+// Tokens are laid out in slices of 16 (the decode kernel runs one launch per
+// slice): token m goes to slice m / 16, `slice_half2` half2 units apart, as
+// token m % 16 of a slice with ceil(tokens in the slice / 8) blocks of 8.
 __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_kernel(
-    const uint16_t* __restrict__ x, int M, int K, __half2* __restrict__ out, float* __restrict__ s_x, int nb,
-    unsigned* __restrict__ zero_words, int zero_count) {
+    const uint16_t* __restrict__ x, int M, int K, __half2* __restrict__ out, float* __restrict__ s_x,
+    int slice_half2, unsigned* __restrict__ zero_words, int zero_count) {
   __shared__ float warp_max[kActClusterBlocks];
   __shared__ float cta_max;
   // The previous kernel may still read the workspace: wait before writing.
@@ -231,9 +222,14 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
   const float s = quant_scale(tmax);
   if (rank == 0 && threadIdx.x == 0) s_x[m] = s;
   if (mine) {
+    const int sl = m >> 4, ml = m & 15;
+    const int in_slice = min(16, M - 16 * sl);
+    const int nb = (in_slice + 7) >> 3;
+    __half2* o = out + int64_t(sl) * slice_half2;
     const int k0 = b * kRotBlock + lane * 8;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[frag_half2_index(m, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], s), quant_code(v[2 * i + 1], s));
+    for (int i = 0; i < 4; ++i)
+      o[frag_half2_index(ml, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], s), quant_code(v[2 * i + 1], s));
   }
   cluster_sync_all();  // no CTA leaves while another may still read its cta_max
 }

@@ -76,7 +76,6 @@ w4a8_status device_state(DeviceState** out) {
       d.err = static_cast<unsigned*>(sym);
       if (allow_smem(rotate_quant_kernel<kActI8Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
-          allow_smem(rotate_quant_kernel<kActF16Frag>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepthSingle, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
@@ -95,11 +94,17 @@ w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK
 
 // ------------------------------------------------------------------ linear workspace
 
-constexpr int kDecodeMaxM = 16;
+// Up to 64 tokens run the decode kernel, in slices of up to 16 tokens (one
+// launch per slice; the weights stream once per slice).  Past that the
+// tensor-core GEMM is faster.
+constexpr int kDecodeSliceM = 16;
+constexpr int kDecodeMaxM = 64;
 
 struct LinearPlan {
   bool decode;
-  int nb;          // decode: token blocks of 8
+  int nb;          // decode: token blocks of 8 of a full slice
+  int slices;      // decode: launches of up to kDecodeSliceM tokens
+  size_t slice_bytes;  // decode: B-fragment bytes of one slice
   size_t off_sx, off_xq, off_cnt, off_slots, total;
   int T, P, C;
 };
@@ -111,14 +116,19 @@ LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
   L.C = int(K / kChunkK);
   L.P = (L.T + kDecTG - 1) / kDecTG;
   if (L.decode) {
-    L.nb = int((M + 7) / 8);
+    const int64_t mslice = M < kDecodeSliceM ? M : kDecodeSliceM;
+    L.nb = int((mslice + 7) / 8);
+    L.slices = int((M + kDecodeSliceM - 1) / kDecodeSliceM);
+    L.slice_bytes = size_t(K) * L.nb * 16;
     L.off_sx = 0;
-    L.off_xq = 256;
-    L.off_cnt = round_up(L.off_xq + size_t(K) * L.nb * 16, 256);
+    L.off_xq = 256;  // s_x: at most 64 floats
+    L.off_cnt = round_up(L.off_xq + L.slice_bytes * L.slices, 256);
     L.off_slots = round_up(L.off_cnt + size_t(L.P) * 4, 256);
-    L.total = round_up(L.off_slots + size_t(2) * kDecMaxCtas * dec_slot_floats(int(M)) * 4, 256);
+    L.total = round_up(L.off_slots + size_t(2) * kDecMaxCtas * dec_slot_floats(int(mslice)) * 4, 256);
   } else {
     L.nb = 0;
+    L.slices = 0;
+    L.slice_bytes = 0;
     L.off_sx = 0;
     L.off_xq = round_up(size_t(M) * 4, 256);
     L.off_cnt = L.off_slots = 0;
@@ -237,7 +247,7 @@ w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_
   DeviceState* d = nullptr;
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   rotate_quant_kernel<kActI8Row><<<unsigned(M), act_threads(K), size_t(K) * 4, static_cast<cudaStream_t>(stream)>>>(
-      x, int(M), int(K), x_q, s_x, 0, nullptr, 0);
+      x, int(M), int(K), x_q, s_x);
   return launch_status();
 }
 
@@ -262,40 +272,46 @@ static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* wo
 static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, int64_t M, int64_t K, int64_t N,
                                  const uint8_t* pk, uint16_t* y, uint8_t* ws, cudaStream_t s, const uint16_t* x) {
   const PackedLayout L = packed_layout(N, K);
-  DecodeParams p;
-  p.x = x;
-  p.units = pk + L.off_units;
-  p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
-  p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
-  p.xfrag = reinterpret_cast<const uint4*>(ws + plan.off_xq);
-  p.s_x = reinterpret_cast<const float*>(ws + plan.off_sx);
-  p.y = y;
-  p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
-  p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
-  p.err = d->err;
-  p.M = int(M);
-  p.N = int(N);
-  p.K = int(K);
-  p.C = plan.C;
-  p.T = plan.T;
-  p.P = plan.P;
-  p.U = plan.P * plan.C;
-  const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
-  p.W = p.U < warps_avail ? p.U : warps_avail;
-  p.R = p.U / p.W;
-  p.Rm = p.U % p.W;
-  const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
-  const size_t smem = dec_smem_bytes(int(M), int(K), M == 1);
-  cudaError_t e;
-  if (x)
-    e = launch_pdl(decode_kernel<1, kDecDepthSingle, true, true>, grid, dim3(kDecThreads), smem, s, p);
-  else if (plan.nb == 1 && M == 1)
-    e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
-  else if (plan.nb == 1)
-    e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(kDecThreads), smem, s, p);
-  else
-    e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(kDecThreads), smem, s, p);
-  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+  for (int sl = 0; sl < plan.slices; ++sl) {
+    const int64_t m0 = int64_t(sl) * kDecodeSliceM;
+    const int64_t ms = M - m0 < kDecodeSliceM ? M - m0 : kDecodeSliceM;
+    DecodeParams p;
+    p.x = x;
+    p.units = pk + L.off_units;
+    p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
+    p.cb = reinterpret_cast<const float*>(pk + L.off_cb);
+    p.xfrag = reinterpret_cast<const uint4*>(ws + plan.off_xq + plan.slice_bytes * sl);
+    p.s_x = reinterpret_cast<const float*>(ws + plan.off_sx) + m0;
+    p.y = y + m0 * N;
+    p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
+    p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
+    p.err = d->err;
+    p.M = int(ms);
+    p.N = int(N);
+    p.K = int(K);
+    p.C = plan.C;
+    p.T = plan.T;
+    p.P = plan.P;
+    p.U = plan.P * plan.C;
+    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
+    p.W = p.U < warps_avail ? p.U : warps_avail;
+    p.R = p.U / p.W;
+    p.Rm = p.U % p.W;
+    const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
+    const size_t smem = dec_smem_bytes(int(ms), int(K), ms == 1);
+    const int nb = int((ms + 7) / 8);
+    cudaError_t e;
+    if (x)
+      e = launch_pdl(decode_kernel<1, kDecDepthSingle, true, true>, grid, dim3(kDecThreads), smem, s, p);
+    else if (ms == 1)
+      e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
+    else if (nb == 1)
+      e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(kDecThreads), smem, s, p);
+    else
+      e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(kDecThreads), smem, s, p);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+  }
+  return W4A8_OK;
 }
 
 w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
@@ -312,12 +328,13 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
     // one cluster of up to 8 CTAs per token (16 blocks of 256 per CTA)
     const unsigned cl = unsigned((K / kRotBlock + kActClusterBlocks - 1) / kActClusterBlocks);
     if (launch_pdl_cluster(rotate_quant_frag_cluster_kernel, dim3(cl, unsigned(M)), dim3(kActClusterThreads), cl, 0,
-                           s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x, plan.nb,
-                           reinterpret_cast<unsigned*>(ws + plan.off_cnt), plan.P) != cudaSuccess)
+                           s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x,
+                           int(plan.slice_bytes / 4), reinterpret_cast<unsigned*>(ws + plan.off_cnt),
+                           plan.P) != cudaSuccess)
       return W4A8_ERR_CUDA;
   } else {
     if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
-                   int(M), int(K), (void*)(ws + plan.off_xq), s_x, 0, (unsigned*)nullptr, 0) != cudaSuccess)
+                   int(M), int(K), (void*)(ws + plan.off_xq), s_x) != cudaSuccess)
       return W4A8_ERR_CUDA;
   }
   return launch_status();
@@ -392,7 +409,7 @@ static std::mutex g_static_scratch_mutex;
 w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, const void* packed, int64_t N,
                                       uint16_t* y, void* stream) {
   if (!x || !packed || !y) return W4A8_ERR_NULL;
-  if (M > kDecodeMaxM || !act_shape_ok(M, K) || !weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (M > kDecodeSliceM || !act_shape_ok(M, K) || !weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
   if (linear_plan(M, K, N).total > kStaticScratchBytes) return W4A8_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
