@@ -204,6 +204,46 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K,
                                       void* stream);
 
 /*
+ * A chain of one-token layers in one persistent launch: a decode step, where
+ * each layer's input is an earlier layer's output (ConvRot card, "Why this
+ * exists": a decode step re-reads every layer's weights for one token).
+ * Layer i computes y_i = w4a8_linear(x_i) for M = 1, with every CTA
+ * rotating and quantising x_i itself; between layers a grid barrier makes
+ * the previous layer's y visible, and each layer's weights are fetched
+ * before that barrier.  Results equal the layer-by-layer w4a8_linear calls
+ * bit for bit.
+ *   layers     host array of n_layers descriptors: packed (w4a8_pack_layout
+ *              buffer for (N, K)), x (device, K bf16), y (device, N bf16).
+ *              An x may be an earlier layer's y (or part of it).  Layers run
+ *              strictly in order (a grid barrier separates them), so a later
+ *              layer may also overwrite a buffer that an earlier one read.
+ * w4a8_chain_plan: check the layers and write their launch table into
+ *   `plan` (device, w4a8_chain_plan_bytes(n) bytes; the call returns once
+ *   the table has been staged) for the given `workspace` (device,
+ *   w4a8_chain_workspace_bytes(layers, n) bytes, owned by the caller).
+ * w4a8_chain_run: run the planned chain on `stream` (capturable in a CUDA
+ *   graph; zeroes the workspace's barrier and counters first).  The launch
+ *   is cooperative (one CTA per SM, all resident); W4A8_ERR_CUDA if the
+ *   device cannot host it.  Two runs sharing a workspace must be ordered.
+ * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA; a grid-barrier wait
+ * that gives up is reported by w4a8_get_device_error as W4A8_ERR_TIMEOUT.
+ */
+typedef struct {
+  const void* packed;
+  int64_t N, K;
+  const uint16_t* x;
+  uint16_t* y;
+} w4a8_chain_layer;
+
+size_t w4a8_chain_plan_bytes(int64_t n_layers);
+size_t w4a8_chain_workspace_bytes(const w4a8_chain_layer* layers, int64_t n_layers);
+w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, void* plan,
+                            size_t plan_bytes, void* workspace, size_t workspace_bytes,
+                            void* stream);
+w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
  * Weight converter on the GPU: fp32 W [N, K] -> the four stored tensors
  * (ConvRot card, "Format": rotate by the group-256 Hadamard, a per-row scale
  * and a per-16 e4m3 scale, 16-level Lloyd-Max codebook, two indices per

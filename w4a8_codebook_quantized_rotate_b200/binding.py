@@ -27,7 +27,14 @@ EXPORTS = (
     "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_status_string",
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
+    "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
 )
+
+
+class ChainLayer(ctypes.Structure):
+    """w4a8_chain_layer: one layer of a chain (device pointers)."""
+    _fields_ = [("packed", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 _lib = None
 
@@ -65,6 +72,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_compare_workspace_bytes": (sz, []),
         "w4a8_compare": (st, [vp, ctypes.c_int32, vp, i64, vp, vp, sz, vp]),
         "w4a8_dense_reference": (st, [vp, i64, i64, vp, i64, vp, vp]),
+        "w4a8_chain_plan_bytes": (sz, [i64]),
+        "w4a8_chain_workspace_bytes": (sz, [vp, i64]),
+        "w4a8_chain_plan": (st, [vp, i64, vp, sz, vp, sz, vp]),
+        "w4a8_chain_run": (st, [vp, i64, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -334,3 +345,37 @@ def verify_layer(w: torch.Tensor, packed: torch.Tensor, x: torch.Tensor, sample_
     rel = lambda c: float((c[0] / c[1]).sqrt()) if c[1] > 0 else float(c[0] > 0)
     return {"fidelity": rel(c1), "fidelity_max_abs": float(c1[2]), "forward": rel(c2),
             "forward_max_abs": float(c2[2]), "fit_rounds": int(fresh["fit_rounds"].item())}
+
+
+def chain_plan(layers, stream=None):
+    """Plan a chain of one-token layers.  ``layers`` is a list of
+    (packed, n, k, x, y): x a bf16 CUDA tensor of k values (may be a view of
+    an earlier layer's y), y a bf16 CUDA tensor of n values.  Returns
+    (plan, workspace, n_layers); the tensors must outlive the runs."""
+    lib = load_library()
+    arr = (ChainLayer * len(layers))()
+    dev = None
+    for i, (packed, n, k, x, y) in enumerate(layers):
+        _cuda(packed, torch.uint8, "packed")
+        _cuda(x, torch.bfloat16, "x")
+        _cuda(y, torch.bfloat16, "y")
+        if x.numel() != k or y.numel() != n:
+            raise ValueError(f"layer {i}: x must hold K and y N values")
+        arr[i] = ChainLayer(packed.data_ptr(), n, k, x.data_ptr(), y.data_ptr())
+        dev = packed.device
+    n_layers = len(layers)
+    plan = torch.empty(lib.w4a8_chain_plan_bytes(n_layers), dtype=torch.uint8, device=dev)
+    ws_bytes = lib.w4a8_chain_workspace_bytes(arr, n_layers)
+    if ws_bytes == 0:
+        raise W4A8Error("w4a8_chain_workspace_bytes", 2)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    _check("w4a8_chain_plan", lib.w4a8_chain_plan(arr, n_layers, plan.data_ptr(), plan.numel(), ws.data_ptr(),
+                                                  ws.numel(), _stream(stream)))
+    return plan, ws, n_layers
+
+
+def chain_run(plan: torch.Tensor, n_layers: int, workspace: torch.Tensor, stream=None) -> None:
+    """Run a planned chain (one persistent launch)."""
+    lib = load_library()
+    _check("w4a8_chain_run", lib.w4a8_chain_run(plan.data_ptr(), n_layers, workspace.data_ptr(), workspace.numel(),
+                                                _stream(stream)))

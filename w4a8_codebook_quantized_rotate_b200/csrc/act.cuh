@@ -61,7 +61,8 @@ __device__ __forceinline__ void fwht8_in_lane(float (&v)[8]) {
 // 256 b + 8 lane .. + 7.  Three butterfly stages inside the lane, five across
 // lanes (shuffles), then the exact 1/16.
 __device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ row, int b, int lane, float (&v)[8]) {
-  const uint4 raw = *reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8);
+  // L2 only: a chain of layers rewrites its activation buffers within one launch
+  const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8));
   const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {

@@ -334,13 +334,18 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 // arithmetic, so the codes and s_x are the same bits).  The rotated row is
 // staged in fp32 below the table as far as it fits (about 63 of the
 // 256-blocks); blocks past that are rotated again when they are quantised.  One launch then makes the whole layer.
-template <int NB, int D, bool SINGLE, bool FUSED = false>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
+//
+// The body is a device function so that a persistent kernel can run a chain
+// of layers with it; `wait_inputs` is where the body waits for what an
+// earlier step wrote (the activations, and the workspace it reuses).
+struct DecWaitPdl {
+  __device__ __forceinline__ void operator()() const { pdl_wait(); }
+};
+
+template <int NB, int D, bool SINGLE, bool FUSED, class Wait>
+__device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& wait_inputs) {
   static_assert(!FUSED || SINGLE, "the fused activation step handles one token");
   extern __shared__ __align__(16) uint8_t dec_smem[];
-  // The next kernel may launch now: it streams its own weights and waits for
-  // this grid's completion before it touches anything this grid writes.
-  pdl_launch_dependents();
   const uint32_t base = smem_u32(dec_smem);
   const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned: bits 8..15 are zero
   const uint32_t xs = lut + 65536u;                   // one token: x staged here (2 K bytes)
@@ -403,7 +408,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
                    "r"(*reinterpret_cast<const uint32_t*>(&h)));
     }
   }
-  pdl_wait();  // activations, scales and counters come from the previous kernel
+  wait_inputs();  // activations, scales and counters come from an earlier step
   int cx = first_c;  // chunk of the next x fragment to load (more than one token)
   if constexpr (FUSED) {
     // Rotate the row (warp per 256-block) and find its absmax.
@@ -617,6 +622,59 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     }
     if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
     dec_epilogue<NB>(acc, p, pr, lane, ep);
+  }
+}
+
+template <int NB, int D, bool SINGLE, bool FUSED = false>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
+  // The next kernel may launch now: it streams its own weights and waits for
+  // this grid's completion before it touches anything this grid writes.
+  pdl_launch_dependents();
+  decode_body<NB, D, SINGLE, FUSED>(p, DecWaitPdl{});
+}
+
+// ---------------------------------------------------------------------------
+// A chain of one-token layers in one persistent launch (a decode step: each
+// layer's input is an earlier layer's output).  Every CTA runs every layer
+// with the fused body; between layers a grid barrier (all CTAs co-resident:
+// cooperative launch) makes the previous layer's y visible.  A layer's
+// weights, table and row scales are fetched before the barrier, since
+// nothing in the chain writes them.  The barrier counter is bounded: a
+// CTA that waits about a second records a timeout and goes on.
+struct DecWaitChain {
+  unsigned* ctr;    // arrivals: CTAs add 1 after each layer
+  unsigned target;  // arrivals that mean the previous layer is complete (0: the first layer)
+  unsigned* err;
+  __device__ __forceinline__ void operator()() const {
+    if (target == 0) {  // the first layer waits for the previous kernel
+      pdl_wait();
+      return;
+    }
+    if (threadIdx.x == 0) {
+      bool done = false;
+      for (uint32_t i = 0; i < (1u << 26) && !done; ++i) {  // an L2 round trip per poll: about a second
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        done = v >= target;
+      }
+      if (!done) record_error(err, kErrTimeout);
+    }
+    __syncthreads();
+  }
+};
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_chain_kernel(const DecodeParams* __restrict__ layers, int n_layers, unsigned* barrier) {
+  pdl_launch_dependents();
+#pragma unroll 1
+  for (int l = 0; l < n_layers; ++l) {
+    const DecodeParams p = layers[l];  // a local copy: the body keeps what it uses in registers
+    decode_body<1, kDecDepthSingle, true, true>(p, DecWaitChain{barrier, unsigned(l) * gridDim.x, p.err});
+    __syncthreads();  // this CTA is done with layer l (its y and workspace writes issued)
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(barrier, 1u);
+    }
   }
 }
 

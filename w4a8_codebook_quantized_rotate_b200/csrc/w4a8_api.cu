@@ -2,6 +2,7 @@
 // and kernel launches.  The declarations, with argument meaning, layout,
 // ownership and error behaviour, are in include/w4a8.h.
 #include <mutex>
+#include <new>
 
 #include "w4a8.h"
 
@@ -78,6 +79,7 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepthSingle, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
+          allow_smem(decode_chain_kernel, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
           allow_smem(decode_kernel<2, kDecDepth2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
@@ -523,6 +525,116 @@ w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const floa
   p.cb = codebook_out;
   convert_row_kernel<0><<<unsigned(N), kCvtThreads, smem, s>>>(p);
   return launch_status();
+}
+
+// ------------------------------------------------------------------ chains of one-token layers
+
+constexpr size_t kChainCounterOff = 256;  // [0, 256): grid-barrier counter
+
+static size_t chain_counter_bytes(const w4a8_chain_layer* layers, int64_t n) {
+  int64_t pmax = 1;
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t p = (layers[i].N / kTileRows + kDecTG - 1) / kDecTG;
+    pmax = p > pmax ? p : pmax;
+  }
+  return round_up(size_t(pmax) * 4, 256);
+}
+
+size_t w4a8_chain_plan_bytes(int64_t n_layers) {
+  return n_layers < 1 ? 0 : round_up(size_t(n_layers) * sizeof(DecodeParams), 256);
+}
+
+size_t w4a8_chain_workspace_bytes(const w4a8_chain_layer* layers, int64_t n_layers) {
+  if (!layers || n_layers < 1) return 0;
+  for (int64_t i = 0; i < n_layers; ++i)
+    if (!weight_shape_ok(layers[i].N, layers[i].K)) return 0;
+  return kChainCounterOff + chain_counter_bytes(layers, n_layers) +
+         round_up(size_t(2) * kDecMaxCtas * dec_slot_floats(1) * 4, 256);
+}
+
+w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, void* plan, size_t plan_bytes,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layers || !plan || !workspace) return W4A8_ERR_NULL;
+  if (n_layers < 1 || n_layers > (int64_t(1) << 20)) return W4A8_ERR_SHAPE;
+  for (int64_t i = 0; i < n_layers; ++i) {
+    const w4a8_chain_layer& L = layers[i];
+    if (!L.packed || !L.x || !L.y) return W4A8_ERR_NULL;
+    if (!weight_shape_ok(L.N, L.K)) return W4A8_ERR_SHAPE;
+    if (!aligned16(L.packed) || !aligned16(L.x) || !aligned16(L.y)) return W4A8_ERR_ALIGN;
+  }
+  if (plan_bytes < w4a8_chain_plan_bytes(n_layers) ||
+      workspace_bytes < w4a8_chain_workspace_bytes(layers, n_layers))
+    return W4A8_ERR_WORKSPACE;
+  if (!aligned16(plan) || !aligned16(workspace)) return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + kChainCounterOff);
+  float* slots = reinterpret_cast<float*>(ws + kChainCounterOff + chain_counter_bytes(layers, n_layers));
+  const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
+  DecodeParams* host = new (std::nothrow) DecodeParams[size_t(n_layers)];
+  if (!host) return W4A8_ERR_SHAPE;
+  for (int64_t i = 0; i < n_layers; ++i) {
+    const w4a8_chain_layer& L = layers[i];
+    const PackedLayout PL = packed_layout(L.N, L.K);
+    const uint8_t* pk = static_cast<const uint8_t*>(L.packed);
+    DecodeParams p{};
+    p.x = L.x;
+    p.units = pk + PL.off_units;
+    p.sch = reinterpret_cast<const float*>(pk + PL.off_sch);
+    p.cb = reinterpret_cast<const float*>(pk + PL.off_cb);
+    p.xfrag = nullptr;
+    p.s_x = nullptr;
+    p.y = L.y;
+    p.slots = slots;
+    p.counters = counters;
+    p.err = d->err;
+    p.M = 1;
+    p.N = int(L.N);
+    p.K = int(L.K);
+    p.C = int(L.K / kChunkK);
+    p.T = int(L.N / kTileRows);
+    p.P = (p.T + kDecTG - 1) / kDecTG;
+    p.U = p.P * p.C;
+    p.W = p.U < warps_avail ? p.U : warps_avail;
+    p.R = p.U / p.W;
+    p.Rm = p.U % p.W;
+    host[i] = p;
+  }
+  // From pageable memory: the call returns once the table has been staged.
+  const cudaError_t e = cudaMemcpyAsync(plan, host, size_t(n_layers) * sizeof(DecodeParams),
+                                        cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
+  delete[] host;
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!plan || !workspace) return W4A8_ERR_NULL;
+  if (n_layers < 1 || n_layers > (int64_t(1) << 20)) return W4A8_ERR_SHAPE;
+  if (workspace_bytes < kChainCounterOff + 256) return W4A8_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the barrier and the split-K counters start at zero
+  const size_t zero = workspace_bytes < kChainCounterOff + (size_t(1) << 16) ? workspace_bytes
+                                                                              : kChainCounterOff + (size_t(1) << 16);
+  if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return W4A8_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas));
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = dec_smem_bytes(1, kMaxK, true);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier can complete
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_chain_kernel, static_cast<const DecodeParams*>(plan),
+                                           int(n_layers), static_cast<unsigned*>(workspace));
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ fidelity checks
