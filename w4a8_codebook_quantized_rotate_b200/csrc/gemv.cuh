@@ -545,24 +545,32 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 
   // ---- level 2: pairs split between warps, reduced by one warp of the CTA
   if (v0 >= v1) return;
-  auto wbeg = [&](int i) -> int {
-    int v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(wbeg_s + uint32_t(i) * 4u));
-    return v;
-  };
+  int wb[kDecWarps + 1];  // the CTA's warp range starts (registers are free after the loop)
+#pragma unroll
+  for (int i = 0; i <= kDecWarps; ++i)
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wb[i]) : "r"(wbeg_s + uint32_t(i) * 4u));
   const int pair_lo = v0 / p.C, pair_hi = (v1 - 1) / p.C;
   for (int pr = pair_lo + wl; pr <= pair_hi; pr += kDecWarps) {
     const int q0 = pr * p.C, q1 = q0 + p.C;  // the pair's units [q0, q1)
     bool whole = false;                       // one warp held all of it (and wrote y)
-    for (int ww = 0; ww < kDecWarps; ++ww) whole = whole || (wbeg(ww) <= q0 && wbeg(ww + 1) >= q1);
+#pragma unroll
+    for (int ww = 0; ww < kDecWarps; ++ww) whole |= (wb[ww] <= q0) & (wb[ww + 1] >= q1);
     if (whole) continue;
+    // the contributors' partials, added in warp order (all loads independent)
     dec_zero<NB>(acc);
+#pragma unroll
     for (int ww = 0; ww < kDecWarps; ++ww) {
-      const int b0 = wbeg(ww), b1 = wbeg(ww + 1);
-      if (b0 < q1 && b1 > q0 && b0 < b1) {  // warp ww holds some of it
-        const uint32_t slot = parts + uint32_t(ww * 2 + (b0 >= q0 ? 0 : 1)) * part_bytes;
-        dec_partial_add_smem<NB>(acc, slot, p.M, lane);
-      }
+      const bool holds = (wb[ww] < q1) & (wb[ww + 1] > q0) & (wb[ww] < wb[ww + 1]);
+      const uint32_t slot = parts + uint32_t(ww * 2 + (wb[ww] >= q0 ? 0 : 1)) * part_bytes;
+      float part[kDecTG][NB][4];
+      dec_zero<NB>(part);
+      dec_partial_add_smem<NB>(part, slot, p.M, lane);
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i)
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[i][j][e] = holds ? acc[i][j][e] + part[i][j][e] : acc[i][j][e];
     }
     if (q0 >= v0 && q1 <= v1) {  // inside this CTA
       dec_epilogue<NB>(acc, p, pr, lane, ep);
