@@ -306,3 +306,26 @@ def test_one_token_single_kernel_equals_two_kernel_path(lib, k):
     assert torch.equal(lib.linear(xt, packed, n, workspace=ws).view(torch.int16), y_one.view(torch.int16))
     wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
     check_linear(y_one.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+@pytest.mark.parametrize("m", [1, 3, 20, 80])
+def test_linear_zero_token_and_zero_rows(lib, m):
+    """An all-zero token gives s_x = 0 and a zero output row; an all-zero
+    weight row gives s_channel = 0 and a zero output column; every path
+    (one-token kernel, decode, sliced decode, GEMM) and the oracle agree."""
+    n, k = 592, 768
+    w = synth.weights(n, k, synth.rng_for(13, 0, "weight"))
+    w[[0, 17, 591]] = 0.0
+    c = O.convert_weight(w)
+    assert c["s_ch"][0] == 0 and c["s_ch"][591] == 0
+    packed = pack(lib, c)
+    bits, x, _ = synth.activations(m, k, synth.rng_for(13, m, "act"), 8)
+    bits[m - 1] = 0
+    x[m - 1] = 0.0
+    y = run_linear(lib, bits, packed, n)
+    assert np.all(y[m - 1] == 0.0)
+    assert np.all(y[:, [0, 17, 591]] == 0.0)
+    if m > 1:
+        wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+        ref = O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"])
+        check_linear(y[: m - 1], ref[: m - 1], x[: m - 1], wmax)
