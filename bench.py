@@ -205,6 +205,24 @@ def cpu_baseline(budget_s: float = 15.0) -> dict:
                       f"{N_DEC} output rows of the M=1 K=5120 layer, {reps} repeats, 1 thread"}
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The maximum of a per-rank figure over the process group (the time of
+    the slowest rank); the value itself when running alone."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(bytes_per_rank_step: float, world: int, steps: int, ms: float) -> float:
+    """Whole-job GB/s: every rank streams its own replica's bytes each step;
+    the time is the slowest rank's."""
+    return world * bytes_per_rank_step * steps / (ms * 1e-3) / 1e9
+
+
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -213,7 +231,7 @@ def run_reference(args) -> None:
     # size each step so that warmup + steps take about two minutes in all
     dt1, _ = time_oracle(q, x, 256, 1)
     per_row = dt1 / 256
-    rows = int(max(16, min(N_DEC, (120.0 / max(1, args.steps + args.warmup)) / per_row)))
+    rows = int(max(16, min(N_DEC, (args.ref_seconds / max(1, args.steps + args.warmup)) / per_row)))
     rows -= rows % 16
     rows = max(rows, 16)
     for _ in range(args.warmup):
@@ -505,6 +523,8 @@ def main() -> None:
     ap.add_argument("--prefill-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the C2/C3/second-prefill lines")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="reference arm: about how long warm-up plus timed steps take in all")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -533,12 +553,8 @@ def main() -> None:
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(v: float) -> float:
+        return max_over_ranks(v, world, dev)
 
     stream = torch.cuda.current_stream()
     peaks = measured_peaks()
@@ -579,9 +595,9 @@ def main() -> None:
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(e0.elapsed_time(e1))
+        ms = ranks_max(e0.elapsed_time(e1))
         ms_step = ms / args.steps
-        value = world * wbytes * args.steps / (ms * 1e-3) / 1e9
+        value = whole_job_rate(wbytes, world, args.steps, ms)
 
         # decode kernel alone: activations prepared once, then back-to-back runs
         B.linear_prepare(x, N_DEC, ws)
@@ -592,7 +608,7 @@ def main() -> None:
         replay_runs()
         g1.record(stream)
         torch.cuda.synchronize()
-        gemv_ms = max_over_ranks(g0.elapsed_time(g1)) / args.steps
+        gemv_ms = ranks_max(g0.elapsed_time(g1)) / args.steps
     dec_clocks = sampler.summary()
     del replay_steps, replay_runs
 
@@ -669,7 +685,7 @@ def main() -> None:
     h1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(h0.elapsed_time(h1)) / e2e_steps
+    e2e_ms = ranks_max(h0.elapsed_time(h1)) / e2e_steps
     del pipe_graphs
     # (b) the same steps issued one by one from Python (host launch cost included)
     h0.record(stream)
@@ -678,7 +694,7 @@ def main() -> None:
     h1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_loop_ms = max_over_ranks(h0.elapsed_time(h1)) / e2e_steps
+    e2e_loop_ms = ranks_max(h0.elapsed_time(h1)) / e2e_steps
     del copies
     torch.cuda.empty_cache()
 
@@ -710,7 +726,7 @@ def main() -> None:
         replay_pre()
         p1.record(stream)
         torch.cuda.synchronize()
-        pre_ms = max_over_ranks(p0.elapsed_time(p1)) / args.prefill_steps
+        pre_ms = ranks_max(p0.elapsed_time(p1)) / args.prefill_steps
         B.linear_prepare(xp, N_PRE, ws_p)
         replay_gemm()
         torch.cuda.synchronize()
@@ -719,7 +735,7 @@ def main() -> None:
         replay_gemm()
         q1.record(stream)
         torch.cuda.synchronize()
-        gemm_ms = max_over_ranks(q0.elapsed_time(q1)) / args.prefill_steps
+        gemm_ms = ranks_max(q0.elapsed_time(q1)) / args.prefill_steps
     del replay_pre, replay_gemm
     pre_clocks = psampler.summary()
 
