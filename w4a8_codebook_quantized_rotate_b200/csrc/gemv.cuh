@@ -15,6 +15,12 @@
 //     and up to 8 tokens; a k16 step is exactly one 16-wide group, so its
 //     fp32 partial is scaled by the group's s_rel in fp32 and accumulated in
 //     fp32;
+//   * for one token the MMA's 8 columns hold 8 groups instead of 8 tokens:
+//     in k16 step s of chunk c only the lanes of column 4 (c & 1) + s carry
+//     x (the B operand is zero elsewhere), so the steps of an even and the
+//     following odd chunk accumulate into one fragment whose columns are
+//     the 8 group partials of each row, and each lane scales its 4 of them
+//     by s_rel in fp32 once per chunk pair (instead of once per step);
 //   * s_x and s_ch scale the final sum in fp32, and y is rounded to bf16.
 //
 // Work split ("stream-K"): a unit is (tile pair p, chunk c), i.e. 32 rows x
@@ -110,6 +116,15 @@ __device__ __forceinline__ void mma_16816z(float (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
+// D += A B.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Per-unit registers: index bytes and group scales of the two tiles, and (for
 // more than one token) the B fragments of the unit's chunk.
 template <int NB, bool SINGLE>
@@ -126,6 +141,11 @@ __device__ __forceinline__ uint4 ld_stream_v4(const uint8_t* p) {
                : "l"(p));
   return v;
 }
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint2 ld_stream_v2(const uint8_t* p) {
   uint2 v;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
@@ -134,12 +154,18 @@ __device__ __forceinline__ uint2 ld_stream_v2(const uint8_t* p) {
 
 // A lane's index words and scale codes of one unit: wp points at the lane's
 // 16 index bytes of tile 0 in the unit, sp at its 8 scale bytes of tile 0.
+// (For one token, sp points at the lane's 4 scale bytes, see dec_compute_one.)
 template <int NB, bool SINGLE>
 __device__ __forceinline__ void dec_load_w(DecStage<NB, SINGLE>& st, const uint8_t* wp, const uint8_t* sp) {
   st.w[0] = ld_stream_v4(wp);
   st.w[1] = ld_stream_v4(wp + kChunkIdxBytes);
-  st.s[0] = ld_stream_v2(sp);
-  st.s[1] = ld_stream_v2(sp + kChunkSrelBytes);
+  if constexpr (SINGLE) {
+    st.s[0].x = ld_stream_u32(sp);
+    st.s[1].x = ld_stream_u32(sp + kChunkSrelBytes);
+  } else {
+    st.s[0] = ld_stream_v2(sp);
+    st.s[1] = ld_stream_v2(sp + kChunkSrelBytes);
+  }
 }
 
 template <int NB, bool SINGLE>
@@ -218,6 +244,45 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, floa
           }
         }
       }
+    }
+  }
+}
+
+// One token, one unit (chunk c): the 32 table lookups, then the 8 MMAs
+// into dm, the fragment shared by the chunk pair (c & ~1, c | 1).  Column n
+// of dm is group n & 3 of chunk (c & ~1) + (n >> 2).  In step s of chunk c
+// only lane (g, t) with g = 4 (c & 1) + s has a non-zero B fragment: x of
+// that group, k = 64 c + 16 s + 2 t (+1) and + 8 (+9), which sit as one
+// 8-byte pair at xb in the staged layout; mpar zeroes it when the chunk's
+// parity is not the lane's (g >> 2) and ms[s] when s != g & 3.
+template <int NB, bool SINGLE>
+__device__ __forceinline__ void dec_compute_one(const DecStage<NB, SINGLE>& st, float (&dm)[kDecTG][4],
+                                                uint32_t lut_lane, uint32_t xb, uint32_t mpar,
+                                                const uint32_t (&ms)[4]) {
+  const uint2 xv = lds64(xb);
+  const uint32_t x0 = xv.x & mpar, x1 = xv.y & mpar;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t a[kDecTG][2][4];
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int s = 2 * h + s2;
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i) {
+        const uint32_t word = s == 0 ? st.w[i].x : s == 1 ? st.w[i].y : s == 2 ? st.w[i].z : st.w[i].w;
+        a[i][s2][0] = lds32(prmt(word, lut_lane, 0x7604u));
+        a[i][s2][1] = lds32(prmt(word, lut_lane, 0x7614u));
+        a[i][s2][2] = lds32(prmt(word, lut_lane, 0x7624u));
+        a[i][s2][3] = lds32(prmt(word, lut_lane, 0x7634u));
+      }
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int s = 2 * h + s2;
+      const uint32_t b0 = x0 & ms[s], b1 = x1 & ms[s];
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i)
+        mma_16816(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1);
     }
   }
 }
@@ -370,7 +435,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   // This lane's index bytes and scale bytes in unit u0; every later unit is
   // kUnitBytes further on.
   const uint8_t* wp = p.units + size_t(u0) * kUnitBytes + lane * 16;
-  const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8;
+  const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8 +
+                      (SINGLE ? 4 * (lane & 1) : 0);
 
   DecStage<NB, SINGLE> st[D];
   // Weights do not depend on the previous kernel: start streaming them first.
@@ -491,10 +557,71 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const uint32_t xs_lane = xs + uint32_t(lane & 3) * 32u;
   float acc[kDecTG][NB][4];
   dec_zero<NB>(acc);
+  // One token: dm is the MMA fragment of the current chunk pair (columns =
+  // its 8 groups), ga the fp32 sums of dm * s_rel (rows g, g + 8 x groups
+  // 2 t, 2 t + 1 of each pair), sr the lane's 4 scale codes of the chunk of
+  // the pair whose groups its columns hold (chunk parity t >> 1): bytes
+  // (row g, group 2 (t & 1)), (row g + 8, same), (row g, group + 1),
+  // (row g + 8, group + 1).
+  float dm[kDecTG][4], ga[kDecTG][4];
+  uint32_t sr[kDecTG], ms[4];
+  const int g_lane = lane >> 2, t_lane = lane & 3;
+#pragma unroll
+  for (int i = 0; i < kDecTG; ++i) {
+    sr[i] = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dm[i][e] = ga[i][e] = 0.f;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) ms[q] = (g_lane & 3) == q ? 0xFFFFFFFFu : 0u;
+  const uint32_t xb_lane = xs_lane + uint32_t(g_lane & 3) * 8u;
+  auto scale_pair = [&]() {
+#pragma unroll
+    for (int i = 0; i < kDecTG; ++i) {
+      const float2 s02 = e4m3x2_to_float2(sr[i]);
+      const float2 s13 = e4m3x2_to_float2(sr[i] >> 16);
+      ga[i][0] = fmaf(dm[i][0], s02.x, ga[i][0]);
+      ga[i][2] = fmaf(dm[i][2], s02.y, ga[i][2]);
+      ga[i][1] = fmaf(dm[i][1], s13.x, ga[i][1]);
+      ga[i][3] = fmaf(dm[i][3], s13.y, ga[i][3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dm[i][e] = 0.f;
+      sr[i] = 0u;
+    }
+  };
+  // Row sums over the lane's group columns and the 4 lanes of a row; the
+  // totals go to acc[i][0][0] (row g) and acc[i][0][2] (row g + 8), token 0.
+  auto finish_rows = [&]() {
+#pragma unroll
+    for (int i = 0; i < kDecTG; ++i) {
+      float r0 = ga[i][0] + ga[i][1], r1 = ga[i][2] + ga[i][3];
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+      acc[i][0][0] = r0;
+      acc[i][0][2] = r1;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ga[i][e] = 0.f;
+    }
+  };
   int cur_pair = first_pair, cur_c = first_c, c_first = first_c;
+  auto compute = [&](const DecStage<NB, SINGLE>& s) {
+    if constexpr (SINGLE) {
+      const uint32_t mpar = (g_lane >> 2) == (cur_c & 1) ? 0xFFFFFFFFu : 0u;
+      dec_compute_one<NB, SINGLE>(s, dm, lut_lane, xb_lane + uint32_t(cur_c) * 128u, mpar, ms);
+      if ((cur_c & 1) == (t_lane >> 1)) {
+#pragma unroll
+        for (int i = 0; i < kDecTG; ++i) sr[i] = s.s[i].x;
+      }
+    } else {
+      dec_compute<NB, SINGLE>(s, acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
+    }
+  };
   // A finished or range-ending pair: write y if this warp covered all of it,
   // else park the partial in shared memory (slot 0: the warp's first pair).
   auto close_pair = [&](int c_last) {
+    if constexpr (SINGLE) finish_rows();
     if (c_first == 0 && c_last == p.C - 1) {
       dec_epilogue<NB>(acc, p, cur_pair, lane, ep);
     } else {
@@ -503,6 +630,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     }
   };
   auto unit_done = [&]() {
+    if constexpr (SINGLE) {
+      if (cur_c & 1) scale_pair();  // an odd chunk completes the pair (C is a multiple of 4)
+    }
     if (++cur_c == p.C) {
       close_pair(p.C - 1);
       dec_zero<NB>(acc);
@@ -523,7 +653,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   for (; ub + 2 * D <= n_units; ub += D) {
 #pragma unroll
     for (int d = 0; d < D; ++d) {
-      dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
+      compute(st[d]);
       refill(st[d], d);
       unit_done();
     }
@@ -535,12 +665,17 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   for (int d2 = 0; d2 < 2 * D; ++d2) {
     const int d = d2 % D;
     if (ub + d2 < n_units) {
-      dec_compute<NB, SINGLE>(st[d], acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
+      compute(st[d]);
       if (ub + d2 + D < n_units) refill(st[d], d2);
       unit_done();
     }
   }
-  if (n_units > 0 && cur_c != 0) close_pair(cur_c - 1);
+  if (n_units > 0 && cur_c != 0) {
+    if constexpr (SINGLE) {
+      if (cur_c & 1) scale_pair();  // the range ended on an even chunk
+    }
+    close_pair(cur_c - 1);
+  }
   __syncthreads();
 
   // ---- level 2: pairs split between warps, reduced by one warp of the CTA
