@@ -48,7 +48,7 @@ constexpr int kDecMaxWarps = kDecMaxCtas * kDecWarps;
 constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
 constexpr int kDecSchRows = 1024;                  // row scales staged in shared memory per CTA
 // Units in flight per warp (register ring depth) per variant.
-constexpr int kDecDepthSingle = 3;                 // one token
+constexpr int kDecDepthSingle = 4;                 // one token (one quad of units, see decode_body)
 constexpr int kDecDepth1 = 3;                      // 2..8 tokens
 constexpr int kDecDepth2 = 2;                      // 9..16 tokens
 
@@ -381,6 +381,65 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 }
 
+// One token: a pair split between warps (levels 2 and 3 of the reduction).
+// Lane l owns row l of the pair (row 16 i + g + 8 h of the partial layout):
+// it adds the contributing warps' partials in warp order, and when the pair
+// also spans other CTAs it parks the CTA's sum in the workspace; the last
+// CTA to arrive (one acquire-release atomic by lane 0) adds the CTAs' sums
+// in CTA order and writes y.
+__device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, int q0, int q1, int v0, int v1,
+                                               const int (&wb)[kDecWarps + 1], uint32_t parts,
+                                               uint32_t part_bytes, int lane, const DecEpi& ep) {
+  float tot = 0.f;
+#pragma unroll
+  for (int ww = 0; ww < kDecWarps; ++ww) {
+    const bool holds = (wb[ww] < q1) & (wb[ww + 1] > q0) & (wb[ww] < wb[ww + 1]);
+    const uint32_t slot = parts + uint32_t(ww * 2 + (wb[ww] >= q0 ? 0 : 1)) * part_bytes;
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(slot + uint32_t(lane) * 4u));
+    tot = holds ? tot + v : tot;
+  }
+  const int row = pr * (kDecTG * 16) + lane;
+  if (!(q0 >= v0 && q1 <= v1)) {
+    // level 3: the pair spans CTAs cf..cl
+    int cf = blockIdx.x, cl = blockIdx.x;
+    while (cf > 0 && dec_cta_begin(cf, p) > q0) --cf;
+    while (dec_cta_begin(cl + 1, p) < q1) ++cl;
+    const int sf = dec_slot_floats(1);
+    p.slots[size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf + lane] = tot;
+    __syncwarp();
+    unsigned old = 0;
+    if (lane == 0)
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + pr) : "memory");
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != unsigned(cl - cf)) return;  // another CTA finishes this pair
+    __syncwarp();  // the other lanes' loads come after lane 0's acquire
+    tot = 0.f;
+    for (int c0 = cf; c0 <= cl; c0 += 4) {
+      float v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int cc = c0 + r;
+        const bool have = cc <= cl;
+        v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin(cc, p) >= q0 ? 0 : 1)) * sf + lane) : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) tot += v[r];
+    }
+    if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
+  }
+  if (row < p.N) {
+    const int rr = row - ep.row0;
+    float sc, sx;
+    if (rr < kDecSchRows)
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(ep.sch + uint32_t(rr) * 4u));
+    else
+      sc = __ldg(p.sch + row);
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sx) : "r"(ep.sx));
+    p.y[row] = __bfloat16_as_ushort(__float2bfloat16_rn(tot * sc * sx));
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Work split ("stream-K"): the P * C units, in the order they lie in memory,
 // are cut into W equal ranges, one per warp; a CTA's 16 warps hold 16
@@ -398,7 +457,10 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 // rotates the bf16 row and quantises it to int8 (the activation kernel's
 // arithmetic, so the codes and s_x are the same bits).  The rotated row is
 // staged in fp32 below the table as far as it fits (about 63 of the
-// 256-blocks); blocks past that are rotated again when they are quantised.  One launch then makes the whole layer.
+// 256-blocks); blocks past that are rotated again when they are quantised.
+// Launched as clusters of two CTAs, each CTA of a pair rotates and
+// quantises every other 256-block and writes its codes into both CTAs'
+// shared memory.  One launch then makes the whole layer.
 //
 // The body is a device function so that a persistent kernel can run a chain
 // of layers with it; `wait_inputs` is where the body waits for what an
@@ -441,11 +503,20 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   DecStage<NB, SINGLE> st[D];
   // Weights do not depend on the previous kernel: start streaming them first.
   // (x for more than one token comes from it, so it is loaded after the wait.)
+  if constexpr (SINGLE) {
+    // one token: slot d holds the next unit u with u % D == d (see the loop below)
 #pragma unroll
-  for (int d = 0; d < D; ++d)
-    if (d < n_units) dec_load_w<NB, SINGLE>(st[d], wp + d * kUnitBytes, sp + d * kUnitBytes);
-  wp += D * kUnitBytes;
-  sp += D * kUnitBytes;
+    for (int d = 0; d < D; ++d) {
+      const int off = ((d - u0) % D + D) % D;  // units from u0 to the first one with residue d
+      if (off < n_units) dec_load_w<NB, SINGLE>(st[d], wp + off * kUnitBytes, sp + off * kUnitBytes);
+    }
+  } else {
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+      if (d < n_units) dec_load_w<NB, SINGLE>(st[d], wp + d * kUnitBytes, sp + d * kUnitBytes);
+    wp += D * kUnitBytes;
+    sp += D * kUnitBytes;
+  }
 
   // The CTA's range, its warps' range starts and its rows' scales (all
   // independent of the previous kernel).
@@ -477,16 +548,23 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   wait_inputs();  // activations, scales and counters come from an earlier step
   int cx = first_c;  // chunk of the next x fragment to load (more than one token)
   if constexpr (FUSED) {
-    // Rotate the row (warp per 256-block) and find its absmax.
+    // Rotate the row (warp per 256-block) and find its absmax.  Launched as
+    // clusters of two CTAs, each CTA of a pair takes every other 256-block:
+    // the pair swaps its maxima and each CTA writes its half of the codes
+    // into both CTAs' shared memory (launched without clusters, a CTA takes
+    // all blocks).
+    const uint32_t crank = cluster_ctarank(), ncta = cluster_nctarank();
     const int nblk = p.K / kRotBlock;
+    const int nown = (nblk - int(crank) + int(ncta) - 1) / int(ncta);  // blocks crank + ncta j
+    const int fit_own = min(nown, fit_blocks);
     float amax = 0.f;
-    for (int b = wl; b < nblk; b += kDecWarps) {
+    for (int j = wl; j < nown; j += kDecWarps) {
       float v[8];
-      rotate_block_lane(p.x, b, lane, v);
+      rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      if (b < fit_blocks) {
-        const uint32_t dst = rot_s + uint32_t(b * kRotBlock + lane * 8) * 4u;
+      if (j < fit_own) {
+        const uint32_t dst = rot_s + uint32_t(j * kRotBlock + lane * 8) * 4u;
         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]),
                      "f"(v[3]));
         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]), "f"(v[6]),
@@ -503,32 +581,43 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       asm volatile("ld.shared.f32 %0, [%1];" : "=f"(m) : "r"(red_s + uint32_t(i) * 4u));
       amax = fmaxf(amax, m);
     }
+    uint32_t peer_xs = 0;
+    if (ncta > 1) {
+      // this CTA's maximum goes to s_x[1]'s slot (one token: unused), read by the partner
+      if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + 4u), "f"(amax));
+      cluster_sync_all();
+      amax = fmaxf(amax, ld_cluster_f32(sx_s + 4u, crank ^ 1u));
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(peer_xs) : "r"(xs), "r"(crank ^ 1u));
+    }
     const float s = quant_scale(amax);
     if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s), "f"(s));
     // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
     // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4; a run
     // of 8 values from k0 (a multiple of 8) covers t = 0..3.
     auto put_codes = [&](int k0, const float (&v)[8]) {
-      const uint32_t dst = xs + uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
+      const uint32_t off = uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const __half2 h = __floats2half2_rn(quant_code(v[2 * t], s), quant_code(v[2 * t + 1], s));
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst + uint32_t(t) * 32u),
-                     "r"(*reinterpret_cast<const uint32_t*>(&h)));
+        const uint32_t hv = *reinterpret_cast<const uint32_t*>(&h);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(xs + off + uint32_t(t) * 32u), "r"(hv));
+        if (ncta > 1) asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(peer_xs + off + uint32_t(t) * 32u), "r"(hv));
       }
     };
-    for (int k0 = threadIdx.x * 8; k0 < fit_blocks * kRotBlock; k0 += kDecThreads * 8) {
+    for (int e = threadIdx.x * 8; e < fit_own * kRotBlock; e += kDecThreads * 8) {
       float v[8];
-      const uint32_t src = rot_s + uint32_t(k0) * 4u;
+      const uint32_t src = rot_s + uint32_t(e) * 4u;
       asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(src));
       asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(src + 16u));
-      put_codes(k0, v);
+      put_codes((int(crank) + int(ncta) * (e >> 8)) * kRotBlock + (e & (kRotBlock - 1)), v);
     }
-    for (int b = fit_blocks + wl; b < nblk; b += kDecWarps) {  // blocks that did not fit: rotate again
+    for (int j = fit_own + wl; j < nown; j += kDecWarps) {  // blocks that did not fit: rotate again
       float v[8];
+      const int b = int(crank) + int(ncta) * j;
       rotate_block_lane(p.x, b, lane, v);
       put_codes(b * kRotBlock + lane * 8, v);
     }
+    if (ncta > 1) cluster_sync_all();  // both halves of the codes are in place; no remote access after this
   } else {
     if (threadIdx.x < p.M)
       asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + threadIdx.x * 4u), "f"(p.s_x[threadIdx.x]));
@@ -630,9 +719,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     }
   };
   auto unit_done = [&]() {
-    if constexpr (SINGLE) {
-      if (cur_c & 1) scale_pair();  // an odd chunk completes the pair (C is a multiple of 4)
-    }
     if (++cur_c == p.C) {
       close_pair(p.C - 1);
       dec_zero<NB>(acc);
@@ -648,6 +734,42 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       if (++cx == p.C) cx = 0;
     }
   };
+  if constexpr (SINGLE) {
+    // Quads: the 4 consecutive units 4 q .. 4 q + 3 are 4 chunks of one tile
+    // pair (C is a multiple of 4), i.e. two chunk pairs.  Slot d holds unit
+    // 4 q + d and is refilled with 4 (q + 1) + d; units outside the warp's
+    // range are skipped (the first and last quads only).  A pair is closed
+    // once per quad at most.
+    static_assert(!SINGLE || D == 4, "one token: the ring is one quad deep");
+    const int q0 = u0 >> 2, q_end = n_units > 0 ? ((u1 - 1) >> 2) + 1 : q0;
+    const uint8_t* wq = wp - size_t(u0 & 3) * kUnitBytes;  // this lane's bytes in unit 4 q0
+    const uint8_t* sq = sp - size_t(u0 & 3) * kUnitBytes;
+    int cq = cur_c & ~3;
+    for (int q = q0; q < q_end; ++q) {
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        const int u = 4 * q + d;
+        if (u >= u0 && u < u1) {
+          cur_c = cq + d;
+          compute(st[d]);
+          if (u + 4 < u1) dec_load_w<NB, SINGLE>(st[d], wq + (4 + d) * kUnitBytes, sq + (4 + d) * kUnitBytes);
+        }
+        if (d & 1) scale_pair();  // chunks cq + d - 1, cq + d
+      }
+      wq += 4 * kUnitBytes;
+      sq += 4 * kUnitBytes;
+      const bool pair_end = cq + 4 == p.C && 4 * q + 4 <= u1;  // the range reaches the pair's last chunk
+      if (pair_end || q == q_end - 1) {
+        close_pair(pair_end ? p.C - 1 : (u1 - 1) - cur_pair * p.C);
+        dec_zero<NB>(acc);
+        ++cur_pair;
+        c_first = 0;
+        cq = 0;
+      } else {
+        cq += 4;
+      }
+    }
+  } else {
   int ub = 0;
   // Full rounds: every stage computes and refills.
   for (; ub + 2 * D <= n_units; ub += D) {
@@ -670,11 +792,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       unit_done();
     }
   }
-  if (n_units > 0 && cur_c != 0) {
-    if constexpr (SINGLE) {
-      if (cur_c & 1) scale_pair();  // the range ended on an even chunk
-    }
-    close_pair(cur_c - 1);
+  if (n_units > 0 && cur_c != 0) close_pair(cur_c - 1);
   }
   __syncthreads();
 
@@ -691,6 +809,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 #pragma unroll
     for (int ww = 0; ww < kDecWarps; ++ww) whole |= (wb[ww] <= q0) & (wb[ww + 1] >= q1);
     if (whole) continue;
+    if constexpr (SINGLE) {
+      dec_reduce_one(p, pr, q0, q1, v0, v1, wb, parts, part_bytes, lane, ep);
+      continue;
+    }
     // the contributors' partials, added in warp order (all loads independent)
     dec_zero<NB>(acc);
 #pragma unroll

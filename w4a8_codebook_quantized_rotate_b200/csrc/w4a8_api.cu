@@ -268,6 +268,14 @@ static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* wo
   return device_state(d);
 }
 
+// One token with K above this: the fused kernel runs as pairs of CTAs that
+// split the activation step (below it the pair's two cluster barriers cost
+// more than the halved rotation saves).
+#ifndef W4A8_DEC_PAIR_K
+#define W4A8_DEC_PAIR_K 8192
+#endif
+constexpr int64_t kDecPairK = W4A8_DEC_PAIR_K;
+
 // Decode launch (M <= 16).  With x given (one token) the kernel also rotates
 // and quantises the token; otherwise it reads what w4a8_linear_prepare left
 // in the workspace.
@@ -303,7 +311,10 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     const size_t smem = dec_smem_bytes(int(ms), int(K), ms == 1);
     const int nb = int((ms + 7) / 8);
     cudaError_t e;
-    if (x)
+    if (x && K > kDecPairK)  // pairs of CTAs share the activation step (an even grid; extra CTAs hold no units)
+      e = launch_pdl_cluster(decode_kernel<1, kDecDepthSingle, true, true>, dim3((grid.x + 1) & ~1u),
+                             dim3(kDecThreads), 2, smem, s, p);
+    else if (x)
       e = launch_pdl(decode_kernel<1, kDecDepthSingle, true, true>, grid, dim3(kDecThreads), smem, s, p);
     else if (ms == 1)
       e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
