@@ -83,10 +83,41 @@ __device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ r
   for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;  // 1/16, exact
 }
 
-// Per-token scale and code: s = amax / 127 (IEEE division), q = clamp(rint(v / s), -127, 127).
+// Per-token scale and code: s = amax / 127 (IEEE division), q = clamp(rint(v / s), -127, 127)
+// with v / s the correctly rounded fp32 quotient.
+//
+// A token's codes take one division each, in every CTA that needs them, so
+// the quotient is formed from the correctly rounded reciprocal r = 1/s and
+// one correction step, q0 = v r, q = q0 + (v - q0 s) r (two fused
+// multiply-adds): P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Develop. 34 (1990), which
+// gives the correctly rounded quotient when r is the correctly rounded
+// reciprocal and nothing overflows or underflows.  The sign of a zero
+// quotient is taken from v.  Scales outside [2^-100, 2^100] use the
+// division itself.
+struct QuantScale {
+  float s;     // amax / 127
+  float r;     // 1 / s, correctly rounded (when fast)
+  bool fast;
+};
 __device__ __forceinline__ float quant_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
-__device__ __forceinline__ float quant_code(float v, float s) {
-  return s > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v, s)), -127.f), 127.f) : 0.f;
+__device__ __forceinline__ QuantScale quant_prepare(float s) {
+  QuantScale q;
+  q.s = s;
+  q.fast = s >= 0x1p-100f && s <= 0x1p100f;
+  q.r = q.fast ? __frcp_rn(s) : 0.f;
+  return q;
+}
+__device__ __forceinline__ float quant_code(float v, const QuantScale& q) {
+  if (!(q.s > 0.f)) return 0.f;
+  float t;
+  if (q.fast) {
+    const float q0 = v * q.r;
+    t = copysignf(fmaf(fmaf(-q0, q.s, v), q.r, q0), v);
+  } else {
+    t = __fdiv_rn(v, q.s);
+  }
+  return fminf(fmaxf(rintf(t), -127.f), 127.f);
 }
 
 template <int OUT>
@@ -121,6 +152,7 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
 #pragma unroll
   for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, warp_max[i]);
   const float s = quant_scale(amax);
+  const QuantScale qs = quant_prepare(s);
   if (threadIdx.x == 0) s_x[m] = s;
   // Quantise 8 consecutive values per thread per step.
   for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
@@ -130,7 +162,7 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
     float q[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      q[i] = quant_code(v[i], s);
+      q[i] = quant_code(v[i], qs);
     }
     if constexpr (OUT == kActI8Row) {
       uint32_t lo = 0, hi = 0;
@@ -221,6 +253,7 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
   float tmax = 0.f;
   for (uint32_t r = 0; r < ncta; ++r) tmax = fmaxf(tmax, ld_cluster_f32(smem_u32(&cta_max), r));
   const float s = quant_scale(tmax);
+  const QuantScale qs = quant_prepare(s);
   if (rank == 0 && threadIdx.x == 0) s_x[m] = s;
   if (mine) {
     const int sl = m >> 4, ml = m & 15;
@@ -230,7 +263,7 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
     const int k0 = b * kRotBlock + lane * 8;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      o[frag_half2_index(ml, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], s), quant_code(v[2 * i + 1], s));
+      o[frag_half2_index(ml, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], qs), quant_code(v[2 * i + 1], qs));
   }
   cluster_sync_all();  // no CTA leaves while another may still read its cta_max
 }

@@ -590,6 +590,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(peer_xs) : "r"(xs), "r"(crank ^ 1u));
     }
     const float s = quant_scale(amax);
+    const QuantScale qs = quant_prepare(s);
     if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s), "f"(s));
     // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
     // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4; a run
@@ -598,7 +599,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       const uint32_t off = uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const __half2 h = __floats2half2_rn(quant_code(v[2 * t], s), quant_code(v[2 * t + 1], s));
+        const __half2 h = __floats2half2_rn(quant_code(v[2 * t], qs), quant_code(v[2 * t + 1], qs));
         const uint32_t hv = *reinterpret_cast<const uint32_t*>(&h);
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(xs + off + uint32_t(t) * 32u), "r"(hv));
         if (ncta > 1) asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(peer_xs + off + uint32_t(t) * 32u), "r"(hv));
