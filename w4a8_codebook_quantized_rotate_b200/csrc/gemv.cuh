@@ -35,6 +35,8 @@
 // adds those and writes y.
 #pragma once
 
+#include <type_traits>
+
 #include "act.cuh"
 #include "common.cuh"
 
@@ -252,15 +254,13 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, floa
 // into dm, the fragment shared by the chunk pair (c & ~1, c | 1).  Column n
 // of dm is group n & 3 of chunk (c & ~1) + (n >> 2).  In step s of chunk c
 // only lane (g, t) with g = 4 (c & 1) + s has a non-zero B fragment: x of
-// that group, k = 64 c + 16 s + 2 t (+1) and + 8 (+9), which sit as one
-// 8-byte pair at xb in the staged layout; mpar zeroes it when the chunk's
-// parity is not the lane's (g >> 2) and ms[s] when s != g & 3.
-template <int NB, bool SINGLE>
+// that group, k = 64 c + 16 s + 2 t (+1) and + 8 (+9).  xv holds that pair
+// for the lane's own chunk of the pair (parity g >> 2), and bm[s] is all
+// ones where step s of this unit's chunk is the lane's.  FIRST: the unit
+// opens the pair, so its first step starts the fragment from zero.
+template <int NB, bool SINGLE, bool FIRST>
 __device__ __forceinline__ void dec_compute_one(const DecStage<NB, SINGLE>& st, float (&dm)[kDecTG][4],
-                                                uint32_t lut_lane, uint32_t xb, uint32_t mpar,
-                                                const uint32_t (&ms)[4]) {
-  const uint2 xv = lds64(xb);
-  const uint32_t x0 = xv.x & mpar, x1 = xv.y & mpar;
+                                                uint32_t lut_lane, uint2 xv, const uint32_t (&bm)[4]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t a[kDecTG][2][4];
@@ -279,10 +279,14 @@ __device__ __forceinline__ void dec_compute_one(const DecStage<NB, SINGLE>& st, 
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
       const int s = 2 * h + s2;
-      const uint32_t b0 = x0 & ms[s], b1 = x1 & ms[s];
+      const uint32_t b0 = xv.x & bm[s], b1 = xv.y & bm[s];
 #pragma unroll
-      for (int i = 0; i < kDecTG; ++i)
-        mma_16816(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1);
+      for (int i = 0; i < kDecTG; ++i) {
+        if (FIRST && s == 0)
+          mma_16816z(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1, 0.f);
+        else
+          mma_16816(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1);
+      }
     }
   }
 }
@@ -455,9 +459,9 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
 //
 // FUSED (one token): the kernel also does the activation step: every CTA
 // rotates the bf16 row and quantises it to int8 (the activation kernel's
-// arithmetic, so the codes and s_x are the same bits).  The rotated row is
-// staged in fp32 below the table as far as it fits (about 63 of the
-// 256-blocks); blocks past that are rotated again when they are quantised.
+// arithmetic, so the codes and s_x are the same bits).  A warp keeps its
+// first few rotated 256-blocks in registers until the row's absmax is known
+// and quantises them from there; blocks past those are rotated again.
 // Launched as clusters of two CTAs, each CTA of a pair rotates and
 // quantises every other 256-block and writes its codes into both CTAs'
 // shared memory.  One launch then makes the whole layer.
@@ -482,9 +486,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
   const uint32_t wbeg_s = sx_s + 64;                                      // warp range starts [17]
   const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
-  const uint32_t rot_s = (base + 15u) & ~15u;                             // FUSED: rotated row, fp32
-  // FUSED: 256-blocks of the rotated row that fit below the table
-  const int fit_blocks = min(p.K / kRotBlock, int((lut - rot_s) / (kRotBlock * 4u)));
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int cta_w0 = blockIdx.x * kDecWarps;
   const int w = cta_w0 + wl;
@@ -523,7 +524,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const int v0 = dec_cta_begin(blockIdx.x, p), v1 = dec_cta_begin(blockIdx.x + 1, p);
   if (lane == 0) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(wl) * 4u), "r"(u0));
-    if (wl == kDecWarps - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + 64u), "r"(v1));
+    if (wl == kDecWarps - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(kDecWarps) * 4u), "r"(v1));
   }
   DecEpi ep;
   ep.sch = sch_s;
@@ -556,20 +557,25 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     const uint32_t crank = cluster_ctarank(), ncta = cluster_nctarank();
     const int nblk = p.K / kRotBlock;
     const int nown = (nblk - int(crank) + int(ncta) - 1) / int(ncta);  // blocks crank + ncta j
-    const int fit_own = min(nown, fit_blocks);
+    // A warp keeps the rotated values of its first kKeep blocks in registers
+    // until the absmax is known; blocks past those are rotated again.
+    constexpr int kKeep = 4;
     float amax = 0.f;
-    for (int j = wl; j < nown; j += kDecWarps) {
+    float vk[kKeep][8];
+#pragma unroll
+    for (int jj = 0; jj < kKeep; ++jj) {
+      const int j = wl + kDecWarps * jj;
+      if (j < nown) {
+        rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, vk[jj]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(vk[jj][i]));
+      }
+    }
+    for (int j = wl + kDecWarps * kKeep; j < nown; j += kDecWarps) {
       float v[8];
       rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      if (j < fit_own) {
-        const uint32_t dst = rot_s + uint32_t(j * kRotBlock + lane * 8) * 4u;
-        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]),
-                     "f"(v[3]));
-        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]), "f"(v[6]),
-                     "f"(v[7]));
-      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -605,14 +611,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
         if (ncta > 1) asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(peer_xs + off + uint32_t(t) * 32u), "r"(hv));
       }
     };
-    for (int e = threadIdx.x * 8; e < fit_own * kRotBlock; e += kDecThreads * 8) {
-      float v[8];
-      const uint32_t src = rot_s + uint32_t(e) * 4u;
-      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(src));
-      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(src + 16u));
-      put_codes((int(crank) + int(ncta) * (e >> 8)) * kRotBlock + (e & (kRotBlock - 1)), v);
+#pragma unroll
+    for (int jj = 0; jj < kKeep; ++jj) {
+      const int j = wl + kDecWarps * jj;
+      if (j < nown) put_codes((int(crank) + int(ncta) * j) * kRotBlock + lane * 8, vk[jj]);
     }
-    for (int j = fit_own + wl; j < nown; j += kDecWarps) {  // blocks that did not fit: rotate again
+    for (int j = wl + kDecWarps * kKeep; j < nown; j += kDecWarps) {
       float v[8];
       const int b = int(crank) + int(ncta) * j;
       rotate_block_lane(p.x, b, lane, v);
@@ -654,29 +658,32 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   // (row g, group 2 (t & 1)), (row g + 8, same), (row g, group + 1),
   // (row g + 8, group + 1).
   float dm[kDecTG][4], ga[kDecTG][4];
-  uint32_t sr[kDecTG], ms[4];
+  uint32_t sr_e[kDecTG], sr_o[kDecTG], bm_e[4], bm_o[4];
   const int g_lane = lane >> 2, t_lane = lane & 3;
 #pragma unroll
   for (int i = 0; i < kDecTG; ++i) {
-    sr[i] = 0u;
+    sr_e[i] = sr_o[i] = 0u;
 #pragma unroll
     for (int e = 0; e < 4; ++e) dm[i][e] = ga[i][e] = 0.f;
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) ms[q] = (g_lane & 3) == q ? 0xFFFFFFFFu : 0u;
-  const uint32_t xb_lane = xs_lane + uint32_t(g_lane & 3) * 8u;
+  for (int q = 0; q < 4; ++q) {
+    bm_e[q] = (g_lane == q) ? 0xFFFFFFFFu : 0u;      // even chunks: lanes g = 0..3
+    bm_o[q] = (g_lane == 4 + q) ? 0xFFFFFFFFu : 0u;  // odd chunks: lanes g = 4..7
+  }
+  // the lane's x pair in the chunk of its parity, relative to the pair's even chunk
+  const uint32_t xb_lane = xs_lane + uint32_t(g_lane & 3) * 8u + uint32_t(g_lane >> 2) * 128u;
+  // Lanes t < 2 hold columns of the even chunk, t >= 2 those of the odd one.
   auto scale_pair = [&]() {
 #pragma unroll
     for (int i = 0; i < kDecTG; ++i) {
-      const float2 s02 = e4m3x2_to_float2(sr[i]);
-      const float2 s13 = e4m3x2_to_float2(sr[i] >> 16);
+      const uint32_t sr = t_lane < 2 ? sr_e[i] : sr_o[i];
+      const float2 s02 = e4m3x2_to_float2(sr);
+      const float2 s13 = e4m3x2_to_float2(sr >> 16);
       ga[i][0] = fmaf(dm[i][0], s02.x, ga[i][0]);
       ga[i][2] = fmaf(dm[i][2], s02.y, ga[i][2]);
       ga[i][1] = fmaf(dm[i][1], s13.x, ga[i][1]);
       ga[i][3] = fmaf(dm[i][3], s13.y, ga[i][3]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dm[i][e] = 0.f;
-      sr[i] = 0u;
     }
   };
   // Row sums over the lane's group columns and the 4 lanes of a row; the
@@ -697,16 +704,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   };
   int cur_pair = first_pair, cur_c = first_c, c_first = first_c;
   auto compute = [&](const DecStage<NB, SINGLE>& s) {
-    if constexpr (SINGLE) {
-      const uint32_t mpar = (g_lane >> 2) == (cur_c & 1) ? 0xFFFFFFFFu : 0u;
-      dec_compute_one<NB, SINGLE>(s, dm, lut_lane, xb_lane + uint32_t(cur_c) * 128u, mpar, ms);
-      if ((cur_c & 1) == (t_lane >> 1)) {
-#pragma unroll
-        for (int i = 0; i < kDecTG; ++i) sr[i] = s.s[i].x;
-      }
-    } else {
-      dec_compute<NB, SINGLE>(s, acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
-    }
+    if constexpr (!SINGLE) dec_compute<NB, SINGLE>(s, acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
   };
   // A finished or range-ending pair: write y if this warp covered all of it,
   // else park the partial in shared memory (slot 0: the warp's first pair).
@@ -741,24 +739,49 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     // 4 q + d and is refilled with 4 (q + 1) + d; units outside the warp's
     // range are skipped (the first and last quads only).  A pair is closed
     // once per quad at most.
-    static_assert(!SINGLE || D == 4, "one token: the ring is one quad deep");
+    static_assert(!SINGLE || D % 4 == 0, "one token: the ring holds whole quads");
+    constexpr int kQ = D / 4;  // quads in flight
     const int q0 = u0 >> 2, q_end = n_units > 0 ? ((u1 - 1) >> 2) + 1 : q0;
-    const uint8_t* wq = wp - size_t(u0 & 3) * kUnitBytes;  // this lane's bytes in unit 4 q0
-    const uint8_t* sq = sp - size_t(u0 & 3) * kUnitBytes;
     int cq = cur_c & ~3;
-    for (int q = q0; q < q_end; ++q) {
+    // One quad q: its units sit in slots 4 r + d (r = q % kQ); each is
+    // refilled with the unit kQ quads further on.
+    auto quad = [&](auto R, int q) {
+      constexpr int r = decltype(R)::value;
+      if (q < q0 || q >= q_end) return;
+      const int lo = u0 - 4 * q, hi = u1 - 4 * q;  // units 4 q + d with lo <= d < hi are the warp's
+      const uint8_t* wq = wp + (4 * q - u0) * kUnitBytes;  // this lane's bytes in unit 4 q
+      const uint8_t* sq = sp + (4 * q - u0) * kUnitBytes;
+      const uint32_t xq = xb_lane + uint32_t(cq) * 128u;
 #pragma unroll
-      for (int d = 0; d < 4; ++d) {
-        const int u = 4 * q + d;
-        if (u >= u0 && u < u1) {
-          cur_c = cq + d;
-          compute(st[d]);
-          if (u + 4 < u1) dec_load_w<NB, SINGLE>(st[d], wq + (4 + d) * kUnitBytes, sq + (4 + d) * kUnitBytes);
+      for (int j = 0; j < 2; ++j) {  // chunk pair (cq + 2 j, cq + 2 j + 1)
+        const uint2 xv = lds64(xq + 256u * j);
+        const int de = 2 * j, dd = 2 * j + 1;
+        if (de >= lo && de < hi) {
+          dec_compute_one<NB, SINGLE, true>(st[4 * r + de], dm, lut_lane, xv, bm_e);
+#pragma unroll
+          for (int i = 0; i < kDecTG; ++i) sr_e[i] = st[4 * r + de].s[i].x;
+          if (de + 4 * kQ < hi)
+            dec_load_w<NB, SINGLE>(st[4 * r + de], wq + (4 * kQ + de) * kUnitBytes, sq + (4 * kQ + de) * kUnitBytes);
+        } else {  // the range starts at the odd chunk
+#pragma unroll
+          for (int i = 0; i < kDecTG; ++i) {
+            sr_e[i] = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dm[i][e] = 0.f;
+          }
         }
-        if (d & 1) scale_pair();  // chunks cq + d - 1, cq + d
+        if (dd >= lo && dd < hi) {
+          dec_compute_one<NB, SINGLE, false>(st[4 * r + dd], dm, lut_lane, xv, bm_o);
+#pragma unroll
+          for (int i = 0; i < kDecTG; ++i) sr_o[i] = st[4 * r + dd].s[i].x;
+          if (dd + 4 * kQ < hi)
+            dec_load_w<NB, SINGLE>(st[4 * r + dd], wq + (4 * kQ + dd) * kUnitBytes, sq + (4 * kQ + dd) * kUnitBytes);
+        } else {  // the range ends at the even chunk
+#pragma unroll
+          for (int i = 0; i < kDecTG; ++i) sr_o[i] = 0u;
+        }
+        scale_pair();
       }
-      wq += 4 * kUnitBytes;
-      sq += 4 * kUnitBytes;
       const bool pair_end = cq + 4 == p.C && 4 * q + 4 <= u1;  // the range reaches the pair's last chunk
       if (pair_end || q == q_end - 1) {
         close_pair(pair_end ? p.C - 1 : (u1 - 1) - cur_pair * p.C);
@@ -769,6 +792,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       } else {
         cq += 4;
       }
+    };
+    for (int q = q0 - q0 % kQ; q < q_end; q += kQ) {
+      quad(std::integral_constant<int, 0>{}, q);
+      if constexpr (kQ > 1) quad(std::integral_constant<int, 1>{}, q + 1);
     }
   } else {
   int ub = 0;
