@@ -42,8 +42,10 @@
 
 namespace w4a8 {
 
-constexpr int kDecWarps = 16;
+constexpr int kDecWarps = 16;                      // one token
 constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecWarpsMulti = 12;                 // 2..16 tokens: fewer warps, more registers each
+__host__ __device__ constexpr int dec_warps(bool single) { return single ? kDecWarps : kDecWarpsMulti; }
 constexpr int kDecTG = 2;                          // tiles (16 rows each) per unit
 constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
 constexpr int kDecMaxWarps = kDecMaxCtas * kDecWarps;
@@ -75,7 +77,7 @@ __host__ __device__ inline int dec_slot_floats(int m) { return kDecTG * 16 * m; 
 // Dynamic shared memory of a launch: table (+ alignment room), one token's
 // activations, and the CTA's per-warp partials.
 __host__ __device__ inline size_t dec_smem_bytes(int m, int k, bool single) {
-  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(kDecWarps) * 2 * dec_slot_floats(m) * 4 +
+  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(dec_warps(single)) * 2 * dec_slot_floats(m) * 4 +
          kDecSchRows * 4 + 64 + 128 + 64;
 }
 
@@ -87,8 +89,9 @@ __device__ __forceinline__ int dec_begin(int w, const DecodeParams& p) {
   return w * p.R + int((unsigned(w) * unsigned(p.Rm)) / unsigned(p.W));
 }
 // CTA c holds warps [16 c, 16 c + 16) (clipped at W).
+template <int WARPS>
 __device__ __forceinline__ int dec_cta_begin(int c, const DecodeParams& p) {
-  return dec_begin(min(c * kDecWarps, p.W), p);
+  return dec_begin(min(c * WARPS, p.W), p);
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -407,8 +410,8 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
   if (!(q0 >= v0 && q1 <= v1)) {
     // level 3: the pair spans CTAs cf..cl
     int cf = blockIdx.x, cl = blockIdx.x;
-    while (cf > 0 && dec_cta_begin(cf, p) > q0) --cf;
-    while (dec_cta_begin(cl + 1, p) < q1) ++cl;
+    while (cf > 0 && dec_cta_begin<kDecWarps>(cf, p) > q0) --cf;
+    while (dec_cta_begin<kDecWarps>(cl + 1, p) < q1) ++cl;
     const int sf = dec_slot_floats(1);
     p.slots[size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf + lane] = tot;
     __syncwarp();
@@ -425,7 +428,7 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
       for (int r = 0; r < 4; ++r) {
         const int cc = c0 + r;
         const bool have = cc <= cl;
-        v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin(cc, p) >= q0 ? 0 : 1)) * sf + lane) : 0.f;
+        v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin<kDecWarps>(cc, p) >= q0 ? 0 : 1)) * sf + lane) : 0.f;
       }
 #pragma unroll
       for (int r = 0; r < 4; ++r) tot += v[r];
@@ -476,18 +479,20 @@ struct DecWaitPdl {
 template <int NB, int D, bool SINGLE, bool FUSED, class Wait>
 __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& wait_inputs) {
   static_assert(!FUSED || SINGLE, "the fused activation step handles one token");
+  constexpr int kW = dec_warps(SINGLE);
+  constexpr int kThr = kW * 32;
   extern __shared__ __align__(16) uint8_t dec_smem[];
   const uint32_t base = smem_u32(dec_smem);
   const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned: bits 8..15 are zero
   const uint32_t xs = lut + 65536u;                   // one token: x staged here (2 K bytes)
   const uint32_t parts = xs + (SINGLE ? uint32_t(p.C) * 128u : 0u);  // [warp][2] partials
   const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
-  const uint32_t sch_s = parts + uint32_t(kDecWarps * 2) * part_bytes;  // row scales
+  const uint32_t sch_s = parts + uint32_t(kW * 2) * part_bytes;  // row scales
   const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
   const uint32_t wbeg_s = sx_s + 64;                                      // warp range starts [17]
   const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const int cta_w0 = blockIdx.x * kDecWarps;
+  const int cta_w0 = blockIdx.x * kW;
   const int w = cta_w0 + wl;
   const int u0 = dec_begin(min(w, p.W), p);
   const int u1 = dec_begin(min(w + 1, p.W), p);
@@ -521,10 +526,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 
   // The CTA's range, its warps' range starts and its rows' scales (all
   // independent of the previous kernel).
-  const int v0 = dec_cta_begin(blockIdx.x, p), v1 = dec_cta_begin(blockIdx.x + 1, p);
+  const int v0 = dec_cta_begin<kW>(blockIdx.x, p), v1 = dec_cta_begin<kW>(blockIdx.x + 1, p);
   if (lane == 0) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(wl) * 4u), "r"(u0));
-    if (wl == kDecWarps - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(kDecWarps) * 4u), "r"(v1));
+    if (wl == kW - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(kW) * 4u), "r"(v1));
   }
   DecEpi ep;
   ep.sch = sch_s;
@@ -532,13 +537,13 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   ep.row0 = (v0 / p.C) * (kDecTG * 16);
   {
     const int rows = min(kDecSchRows, min(p.N, (v1 > v0 ? (v1 - 1) / p.C + 1 : 0) * kDecTG * 16) - ep.row0);
-    for (int i = threadIdx.x; i < rows; i += kDecThreads)
+    for (int i = threadIdx.x; i < rows; i += kThr)
       asm volatile("st.shared.f32 [%0], %1;" ::"r"(sch_s + uint32_t(i) * 4u), "f"(__ldg(p.sch + ep.row0 + i)));
   }
   // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
   {
     const float level = p.cb[lane & 15];
-    for (int b = wl; b < 256; b += kDecWarps) {
+    for (int b = wl; b < 256; b += kW) {
       const float lo = __shfl_sync(0xffffffffu, level, b & 15);
       const float hi = __shfl_sync(0xffffffffu, level, b >> 4);
       const __half2 h = __floats2half2_rn(lo, hi);
@@ -564,14 +569,14 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     float vk[kKeep][8];
 #pragma unroll
     for (int jj = 0; jj < kKeep; ++jj) {
-      const int j = wl + kDecWarps * jj;
+      const int j = wl + kW * jj;
       if (j < nown) {
         rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, vk[jj]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(vk[jj][i]));
       }
     }
-    for (int j = wl + kDecWarps * kKeep; j < nown; j += kDecWarps) {
+    for (int j = wl + kW * kKeep; j < nown; j += kW) {
       float v[8];
       rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, v);
 #pragma unroll
@@ -582,7 +587,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(red_s + uint32_t(wl) * 4u), "f"(amax));
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < kDecWarps; ++i) {
+    for (int i = 0; i < kW; ++i) {
       float m;
       asm volatile("ld.shared.f32 %0, [%1];" : "=f"(m) : "r"(red_s + uint32_t(i) * 4u));
       amax = fmaxf(amax, m);
@@ -613,10 +618,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     };
 #pragma unroll
     for (int jj = 0; jj < kKeep; ++jj) {
-      const int j = wl + kDecWarps * jj;
+      const int j = wl + kW * jj;
       if (j < nown) put_codes((int(crank) + int(ncta) * j) * kRotBlock + lane * 8, vk[jj]);
     }
-    for (int j = wl + kDecWarps * kKeep; j < nown; j += kDecWarps) {
+    for (int j = wl + kW * kKeep; j < nown; j += kW) {
       float v[8];
       const int b = int(crank) + int(ncta) * j;
       rotate_block_lane(p.x, b, lane, v);
@@ -629,7 +634,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     if constexpr (SINGLE) {
       // token 0's B fragments: per chunk, lanes t = 0..3 of the fragment layout (128 bytes)
       const uint8_t* src = reinterpret_cast<const uint8_t*>(p.xfrag);
-      for (int e = threadIdx.x; e < p.C * 8; e += kDecThreads) {
+      for (int e = threadIdx.x; e < p.C * 8; e += kThr) {
         const int c = e >> 3, qq = e & 7;
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + size_t(c) * 1024 + qq * 16));
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + uint32_t(c) * 128u + uint32_t(qq) * 16u),
@@ -826,16 +831,16 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 
   // ---- level 2: pairs split between warps, reduced by one warp of the CTA
   if (v0 >= v1) return;
-  int wb[kDecWarps + 1];  // the CTA's warp range starts (registers are free after the loop)
+  int wb[kW + 1];  // the CTA's warp range starts (registers are free after the loop)
 #pragma unroll
-  for (int i = 0; i <= kDecWarps; ++i)
+  for (int i = 0; i <= kW; ++i)
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wb[i]) : "r"(wbeg_s + uint32_t(i) * 4u));
   const int pair_lo = v0 / p.C, pair_hi = (v1 - 1) / p.C;
-  for (int pr = pair_lo + wl; pr <= pair_hi; pr += kDecWarps) {
+  for (int pr = pair_lo + wl; pr <= pair_hi; pr += kW) {
     const int q0 = pr * p.C, q1 = q0 + p.C;  // the pair's units [q0, q1)
     bool whole = false;                       // one warp held all of it (and wrote y)
 #pragma unroll
-    for (int ww = 0; ww < kDecWarps; ++ww) whole |= (wb[ww] <= q0) & (wb[ww + 1] >= q1);
+    for (int ww = 0; ww < kW; ++ww) whole |= (wb[ww] <= q0) & (wb[ww + 1] >= q1);
     if (whole) continue;
     if constexpr (SINGLE) {
       dec_reduce_one(p, pr, q0, q1, v0, v1, wb, parts, part_bytes, lane, ep);
@@ -844,7 +849,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     // the contributors' partials, added in warp order (all loads independent)
     dec_zero<NB>(acc);
 #pragma unroll
-    for (int ww = 0; ww < kDecWarps; ++ww) {
+    for (int ww = 0; ww < kW; ++ww) {
       const bool holds = (wb[ww] < q1) & (wb[ww + 1] > q0) & (wb[ww] < wb[ww + 1]);
       const uint32_t slot = parts + uint32_t(ww * 2 + (wb[ww] >= q0 ? 0 : 1)) * part_bytes;
       float part[kDecTG][NB][4];
@@ -863,8 +868,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     }
     // ---- level 3: the pair spans CTAs cf..cl; park this CTA's partial in the workspace
     int cf = blockIdx.x, cl = blockIdx.x;
-    while (cf > 0 && dec_cta_begin(cf, p) > q0) --cf;
-    while (dec_cta_begin(cl + 1, p) < q1) ++cl;
+    while (cf > 0 && dec_cta_begin<kW>(cf, p) > q0) --cf;
+    while (dec_cta_begin<kW>(cl + 1, p) < q1) ++cl;
     const int sf = dec_slot_floats(p.M);
     const int g = lane >> 2, t = lane & 3;
     float* mine = p.slots + size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf;
@@ -893,7 +898,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       for (int r = 0; r < kMaxCtaParts; ++r) {
         const int cc = c0 + r;
         const bool have = cc <= cl;
-        const float* src = p.slots + size_t(cc * 2 + (have && dec_cta_begin(cc, p) >= q0 ? 0 : 1)) * sf;
+        const float* src = p.slots + size_t(cc * 2 + (have && dec_cta_begin<kW>(cc, p) >= q0 ? 0 : 1)) * sf;
 #pragma unroll
         for (int i = 0; i < kDecTG; ++i)
 #pragma unroll
@@ -919,7 +924,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 }
 
 template <int NB, int D, bool SINGLE, bool FUSED = false>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(dec_warps(SINGLE) * 32, 1) decode_kernel(const DecodeParams p) {
   // The next kernel may launch now: it streams its own weights and waits for
   // this grid's completion before it touches anything this grid writes.
   pdl_launch_dependents();

@@ -303,11 +303,12 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     p.T = plan.T;
     p.P = plan.P;
     p.U = plan.P * plan.C;
-    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
+    const int wpc = dec_warps(ms == 1);  // warps per CTA of this variant
+    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * wpc;
     p.W = p.U < warps_avail ? p.U : warps_avail;
     p.R = p.U / p.W;
     p.Rm = p.U % p.W;
-    const dim3 grid((p.W + kDecWarps - 1) / kDecWarps);
+    const dim3 grid((p.W + wpc - 1) / wpc);
     const size_t smem = dec_smem_bytes(int(ms), int(K), ms == 1);
     const int nb = int((ms + 7) / 8);
     cudaError_t e;
@@ -319,9 +320,9 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     else if (ms == 1)
       e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
     else if (nb == 1)
-      e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(kDecThreads), smem, s, p);
+      e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(wpc * 32), smem, s, p);
     else
-      e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(kDecThreads), smem, s, p);
+      e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(wpc * 32), smem, s, p);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
   }
   return W4A8_OK;
