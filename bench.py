@@ -779,7 +779,7 @@ def main() -> None:
             "launch": "timed steps replayed from CUDA graphs (1 kernel per step, programmatic dependent launch)",
         },
         "roofline": {
-            "kernel": "decode_kernel<1,3,1,1> (M=1, rotate + quantise fused)",
+            "kernel": "decode_kernel<1,4,1,1> (M=1, rotate + quantise fused)",
             "bound": "hbm", "achieved": step_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": step_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
             "traffic": profiled_traffic("decode_kernel_fused", ["gemv.cuh", "act.cuh", "common.cuh"]),
@@ -787,7 +787,7 @@ def main() -> None:
             "note": "the step is this one kernel, so its launch duration is the step time",
         },
         "decode_run_only": {
-            "kernel": "decode_kernel<1,3,1,0> (activations prepared once, runs back to back)",
+            "kernel": "decode_kernel<1,4,1,0> (activations prepared once, runs back to back)",
             "achieved": achieved, "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
             "us_per_launch": gemv_ms * 1e3,
         },
