@@ -289,9 +289,10 @@ def test_prepare_once_run_several_layers(lib, m):
 @pytest.mark.parametrize("k", [5120, 15872, 16128, 17408, 32768])
 def test_one_token_single_kernel_equals_two_kernel_path(lib, k):
     """For one token, w4a8_linear is one kernel that rotates and quantises the
-    token itself (K > ~16K: the blocks that do not fit in shared memory are
-    rotated a second time); it must give the same bits as the activation
-    kernel followed by the decode kernel, and match the oracle."""
+    token itself (above K = 8192 as pairs of CTAs that split the rotation;
+    past 64 blocks a warp rotates some blocks a second time); it must give
+    the same bits as the activation kernel followed by the decode kernel,
+    and match the oracle."""
     n = 592
     c = O.convert_weight(synth.weights(n, k, synth.rng_for(70, k, "weight")), sample_cap=2**16)
     packed = pack(lib, c)
@@ -304,6 +305,29 @@ def test_one_token_single_kernel_equals_two_kernel_path(lib, k):
     assert torch.equal(y_one.view(torch.int16), y_two.view(torch.int16))
     # and again through the same workspace (its split-K counters were left at zero)
     assert torch.equal(lib.linear(xt, packed, n, workspace=ws).view(torch.int16), y_one.view(torch.int16))
+    wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
+    check_linear(y_one.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
+@pytest.mark.parametrize("n,k", [(16, 8448), (48, 16640), (272, 8960), (16, 256), (1040, 8448)])
+def test_one_token_small_grids_and_long_pairs(lib, n, k):
+    """One token on shapes whose warp count is not a multiple of the CTA size:
+    the CTA-pair launch rounds the grid up to an even count (the extra CTA
+    holds no units), and with few rows and a long K a single row pair spans
+    many CTAs, so its last CTA adds many workspace partials.  Same bits as
+    the two-kernel path, repeatable through one workspace, and the oracle's
+    values within the bars."""
+    c = O.convert_weight(synth.weights(n, k, synth.rng_for(71, n + k, "weight")), sample_cap=2**16)
+    packed = pack(lib, c)
+    bits, x, _ = synth.activations(1, k, synth.rng_for(11, n + k, "act"), max(1, k // 100))
+    xt = bf16(bits)
+    ws = lib.linear_workspace(1, k, n, "cuda")
+    y_one = lib.linear(xt, packed, n, workspace=ws)
+    y_again = lib.linear(xt, packed, n, workspace=ws)
+    assert torch.equal(y_one.view(torch.int16), y_again.view(torch.int16))
+    lib.linear_prepare(xt, n, ws)
+    y_two = lib.linear_run(1, k, packed, n, ws)
+    assert torch.equal(y_one.view(torch.int16), y_two.view(torch.int16))
     wmax = float(np.abs(O.dequant(c["idx"], c["s_rel"], c["s_ch"], c["cb"])).max())
     check_linear(y_one.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
 

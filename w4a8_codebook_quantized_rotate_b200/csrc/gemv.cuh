@@ -48,7 +48,6 @@ constexpr int kDecWarpsMulti = 12;                 // 2..16 tokens: fewer warps,
 __host__ __device__ constexpr int dec_warps(bool single) { return single ? kDecWarps : kDecWarpsMulti; }
 constexpr int kDecTG = 2;                          // tiles (16 rows each) per unit
 constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
-constexpr int kDecMaxWarps = kDecMaxCtas * kDecWarps;
 constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
 constexpr int kDecSchRows = 1024;                  // row scales staged in shared memory per CTA
 // Units in flight per warp (register ring depth) per variant.
@@ -658,10 +657,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   dec_zero<NB>(acc);
   // One token: dm is the MMA fragment of the current chunk pair (columns =
   // its 8 groups), ga the fp32 sums of dm * s_rel (rows g, g + 8 x groups
-  // 2 t, 2 t + 1 of each pair), sr the lane's 4 scale codes of the chunk of
-  // the pair whose groups its columns hold (chunk parity t >> 1): bytes
-  // (row g, group 2 (t & 1)), (row g + 8, same), (row g, group + 1),
-  // (row g + 8, group + 1).
+  // 2 t, 2 t + 1 of each pair).  sr_e / sr_o hold the lane's 4 scale codes
+  // of the pair's even / odd chunk, bytes (row g, group 2 (t & 1)),
+  // (row g + 8, same), (row g, group + 1), (row g + 8, group + 1); lanes
+  // t < 2 apply the even chunk's, t >= 2 the odd one's.  bm_e / bm_o: the
+  // lane's B-fragment masks per k16 step for even / odd chunks.
   float dm[kDecTG][4], ga[kDecTG][4];
   uint32_t sr_e[kDecTG], sr_o[kDecTG], bm_e[4], bm_o[4];
   const int g_lane = lane >> 2, t_lane = lane & 3;
@@ -708,7 +708,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     }
   };
   int cur_pair = first_pair, cur_c = first_c, c_first = first_c;
-  auto compute = [&](const DecStage<NB, SINGLE>& s) {
+  auto compute = [&](const DecStage<NB, SINGLE>& s) {  // 2..16 tokens (one token: the quad loop below)
     if constexpr (!SINGLE) dec_compute<NB, SINGLE>(s, acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
   };
   // A finished or range-ending pair: write y if this warp covered all of it,
@@ -740,8 +740,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   };
   if constexpr (SINGLE) {
     // Quads: the 4 consecutive units 4 q .. 4 q + 3 are 4 chunks of one tile
-    // pair (C is a multiple of 4), i.e. two chunk pairs.  Slot d holds unit
-    // 4 q + d and is refilled with 4 (q + 1) + d; units outside the warp's
+    // pair (C is a multiple of 4), i.e. two chunk pairs.  The ring holds
+    // kQ = D / 4 quads: unit 4 q + d sits in slot 4 (q mod kQ) + d and the
+    // slot is refilled with unit 4 (q + kQ) + d.  Units outside the warp's
     // range are skipped (the first and last quads only).  A pair is closed
     // once per quad at most.
     static_assert(!SINGLE || D % 4 == 0, "one token: the ring holds whole quads");
