@@ -15,6 +15,8 @@
 // staged in shared memory until the row maximum is known.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace w4a8 {
@@ -108,16 +110,16 @@ __device__ __forceinline__ QuantScale quant_prepare(float s) {
   q.r = q.fast ? __frcp_rn(s) : 0.f;
   return q;
 }
+// FAST: the scale is in the reciprocal's range (QuantScale::fast); callers
+// branch on it once per token, so each loop carries one form only.
+template <bool FAST>
 __device__ __forceinline__ float quant_code(float v, const QuantScale& q) {
-  if (!(q.s > 0.f)) return 0.f;
-  float t;
-  if (q.fast) {
+  if constexpr (FAST) {
     const float q0 = v * q.r;
-    t = copysignf(fmaf(fmaf(-q0, q.s, v), q.r, q0), v);
+    return fminf(fmaxf(rintf(copysignf(fmaf(fmaf(-q0, q.s, v), q.r, q0), v)), -127.f), 127.f);
   } else {
-    t = __fdiv_rn(v, q.s);
+    return q.s > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v, q.s)), -127.f), 127.f) : 0.f;
   }
-  return fminf(fmaxf(rintf(t), -127.f), 127.f);
 }
 
 template <int OUT>
@@ -155,31 +157,37 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
   const QuantScale qs = quant_prepare(s);
   if (threadIdx.x == 0) s_x[m] = s;
   // Quantise 8 consecutive values per thread per step.
-  for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
-    const float4 a = *reinterpret_cast<const float4*>(xr + k0);
-    const float4 c = *reinterpret_cast<const float4*>(xr + k0 + 4);
-    const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-    float q[8];
+  auto quantise = [&](auto fast) {
+    for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
+      const float4 a = *reinterpret_cast<const float4*>(xr + k0);
+      const float4 c = *reinterpret_cast<const float4*>(xr + k0 + 4);
+      const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      q[i] = quant_code(v[i], qs);
-    }
-    if constexpr (OUT == kActI8Row) {
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo |= (uint32_t(int(q[i])) & 0xFFu) << (8 * i);
-        hi |= (uint32_t(int(q[i + 4])) & 0xFFu) << (8 * i);
+      for (int i = 0; i < 8; ++i) {
+        q[i] = quant_code<decltype(fast)::value>(v[i], qs);
       }
-      *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + int64_t(m) * K + k0) = make_uint2(lo, hi);
-    } else {
-      __half2 h[4];
+      if constexpr (OUT == kActI8Row) {
+        uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
-      *reinterpret_cast<uint4*>(static_cast<__half*>(out) + int64_t(m) * K + k0) =
-          *reinterpret_cast<uint4*>(h);
+        for (int i = 0; i < 4; ++i) {
+          lo |= (uint32_t(int(q[i])) & 0xFFu) << (8 * i);
+          hi |= (uint32_t(int(q[i + 4])) & 0xFFu) << (8 * i);
+        }
+        *reinterpret_cast<uint2*>(static_cast<int8_t*>(out) + int64_t(m) * K + k0) = make_uint2(lo, hi);
+      } else {
+        __half2 h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(q[2 * i], q[2 * i + 1]);
+        *reinterpret_cast<uint4*>(static_cast<__half*>(out) + int64_t(m) * K + k0) =
+            *reinterpret_cast<uint4*>(h);
+      }
     }
-  }
+  };
+  if (qs.fast)
+    quantise(std::true_type{});
+  else
+    quantise(std::false_type{});
 }
 
 // The decode operand for a few tokens, one token per thread-block cluster:
@@ -261,9 +269,17 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
     const int nb = (in_slice + 7) >> 3;
     __half2* o = out + int64_t(sl) * slice_half2;
     const int k0 = b * kRotBlock + lane * 8;
+    auto put = [&](auto fast) {
+      constexpr bool kFast = decltype(fast)::value;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[frag_half2_index(ml, k0 + 2 * i, nb)] = __floats2half2_rn(quant_code(v[2 * i], qs), quant_code(v[2 * i + 1], qs));
+      for (int i = 0; i < 4; ++i)
+        o[frag_half2_index(ml, k0 + 2 * i, nb)] =
+            __floats2half2_rn(quant_code<kFast>(v[2 * i], qs), quant_code<kFast>(v[2 * i + 1], qs));
+    };
+    if (qs.fast)
+      put(std::true_type{});
+    else
+      put(std::false_type{});
   }
   cluster_sync_all();  // no CTA leaves while another may still read its cta_max
 }

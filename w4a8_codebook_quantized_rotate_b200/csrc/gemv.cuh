@@ -605,27 +605,34 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
     // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4; a run
     // of 8 values from k0 (a multiple of 8) covers t = 0..3.
-    auto put_codes = [&](int k0, const float (&v)[8]) {
+    auto put_codes = [&](auto fast, int k0, const float (&v)[8]) {
+      constexpr bool kFast = decltype(fast)::value;
       const uint32_t off = uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const __half2 h = __floats2half2_rn(quant_code(v[2 * t], qs), quant_code(v[2 * t + 1], qs));
+        const __half2 h = __floats2half2_rn(quant_code<kFast>(v[2 * t], qs), quant_code<kFast>(v[2 * t + 1], qs));
         const uint32_t hv = *reinterpret_cast<const uint32_t*>(&h);
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(xs + off + uint32_t(t) * 32u), "r"(hv));
         if (ncta > 1) asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(peer_xs + off + uint32_t(t) * 32u), "r"(hv));
       }
     };
+    auto quantise = [&](auto fast) {
 #pragma unroll
-    for (int jj = 0; jj < kKeep; ++jj) {
-      const int j = wl + kW * jj;
-      if (j < nown) put_codes((int(crank) + int(ncta) * j) * kRotBlock + lane * 8, vk[jj]);
-    }
-    for (int j = wl + kW * kKeep; j < nown; j += kW) {
-      float v[8];
-      const int b = int(crank) + int(ncta) * j;
-      rotate_block_lane(p.x, b, lane, v);
-      put_codes(b * kRotBlock + lane * 8, v);
-    }
+      for (int jj = 0; jj < kKeep; ++jj) {
+        const int j = wl + kW * jj;
+        if (j < nown) put_codes(fast, (int(crank) + int(ncta) * j) * kRotBlock + lane * 8, vk[jj]);
+      }
+      for (int j = wl + kW * kKeep; j < nown; j += kW) {
+        float v[8];
+        const int b = int(crank) + int(ncta) * j;
+        rotate_block_lane(p.x, b, lane, v);
+        put_codes(fast, b * kRotBlock + lane * 8, v);
+      }
+    };
+    if (qs.fast)
+      quantise(std::true_type{});
+    else
+      quantise(std::false_type{});
     if (ncta > 1) cluster_sync_all();  // both halves of the codes are in place; no remote access after this
   } else {
     if (threadIdx.x < p.M)
