@@ -28,11 +28,10 @@ enum ActOut : int {
 
 constexpr int kActMaxThreads = 1024;
 
-// Threads per token: one warp per 256-block, between 256 and 1024.
-__host__ __device__ inline int act_threads(int64_t K) {
-  const int64_t t = 32 * (K / kRotBlock);
-  return int(t < 256 ? 256 : (t > kActMaxThreads ? kActMaxThreads : t));
-}
+// Threads per token: 8 warps (a warp takes every 8th 256-block).  Fewer
+// threads than blocks lets more tokens share an SM (measured: 29 vs 38 us
+// for 4096 tokens at K = 5120 against one warp per block).
+__host__ __device__ inline int act_threads(int64_t) { return 256; }
 
 // Index (in half2 units) of element (m, k) in the decode B-fragment layout:
 // [chunk][n8 block j][lane 32][8 half2], lane = 4 (m % 8) + t, half2
