@@ -304,6 +304,55 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
     return {"workload": f"K={k} N={n}, 8 weight copies cycled, one w4a8_linear per call", "by_m": out}
 
 
+def measure_c1_rate(B, synth, torch, dev, rank, stream, steps=400, copies=4):
+    """The one-token layer at K=5120 with N = 17408 x {1, 2, 4, 8} (4 weight
+    copies cycled, all larger than L2 together): the time per extra 50.2 MB is
+    the streaming loop's rate, and the line through the points at N = 0 is the
+    per-call cost that does not scale with the weights (the wait for the
+    previous grid, the activation step, the tail)."""
+    k = 5120
+    pts = []
+    for mult in (1, 2, 4, 8):
+        n = 17408 * mult
+        ws_ = []
+        for c in range(copies):
+            q = synth.quantized_format_device(n, k, seed=5000 * (rank + 1) + 10 * mult + c, device=dev)
+            ws_.append(B.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"]))
+            del q
+        g = torch.Generator(device=dev)
+        g.manual_seed(500 + mult)
+        x = torch.randn((1, k), generator=g, device=dev).to(torch.bfloat16)
+        ws = B.linear_workspace(1, k, n, dev)
+        y = torch.empty((1, n), dtype=torch.bfloat16, device=dev)
+        st = max(40, steps // mult)
+
+        def step(i):
+            B.linear(x, ws_[i % copies], n, workspace=ws, out=y)
+
+        for i in range(5):
+            step(i)
+        replay = graph_loop(step, st, stream)
+        replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pts.append((weight_bytes(n, k), e0.elapsed_time(e1) * 1e3 / st))
+        del replay, ws_
+        torch.cuda.empty_cache()
+    xs = [b for b, _ in pts]
+    ys = [t for _, t in pts]
+    xm, ym = sum(xs) / len(xs), sum(ys) / len(ys)
+    slope = sum((a - xm) * (b - ym) for a, b in zip(xs, ys)) / sum((a - xm) ** 2 for a in xs)  # us per byte
+    return {"workload": "M=1 K=5120, N = 17408 x {1,2,4,8}, 4 weight copies cycled, one w4a8_linear per call",
+            "us_per_call": {str(17408 * m): round(t, 3) for m, (_, t) in zip((1, 2, 4, 8), pts)},
+            "stream_GBs": 1e-3 / slope,
+            "fixed_us": ym - slope * xm,
+            "how": "least-squares line of time per call against weight bytes"}
+
+
 def measure_c3(B, synth, torch, dev, rank, stream, steps, warmup):
     """Decode step of a 62-block stack of projections, M=1, all weights
     distinct and resident.  Per block the projections run as a chain:
@@ -743,6 +792,7 @@ def main() -> None:
     extra = {}
     if not args.no_extra:
         extra["c2_down_proj"] = measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup)
+        extra["c1_streaming_rate"] = measure_c1_rate(B, synth, torch, dev, rank, stream)
         extra["c3_decode_step"] = measure_c3(B, synth, torch, dev, rank, stream, 20, 3)
         extra["c4_prefill_8192"] = measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3)
         extra["weight_converter"] = measure_converter(B, torch, dev, rank, stream)

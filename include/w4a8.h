@@ -120,13 +120,15 @@ w4a8_status w4a8_rotate_quant_act(const uint16_t* x, int64_t M, int64_t K,
 /*
  * Bytes of device workspace w4a8_linear needs for (M, K, N), or 0 if the
  * shape breaks the rules.  The workspace holds the quantised activations,
- * their scales, the split-K partial sums and the split-K arrival counters.
- * Fill a new workspace with zeros before its first use (for example
- * cudaMemsetAsync): the one-token path of w4a8_linear needs the counters at
- * zero when it starts, and every completed call leaves them at zero again
- * (w4a8_linear_prepare also clears them).  After a call that reported
- * W4A8_ERR_TIMEOUT, zero the workspace again.  Everything else in it is
- * scratch between calls.
+ * their scales, the split-K partial sums and, at its start, the words that
+ * join partial sums across CTAs (arrival counters, exchange words).  Fill a
+ * new workspace with zeros before its first use (for example
+ * cudaMemsetAsync): the decode kernel needs those words at zero when it
+ * starts, and every completed call leaves them at zero again.  They sit at
+ * the same offsets, with the same size, for every shape and nothing else
+ * writes there, so one workspace may serve calls of different shapes.
+ * After a call that reported W4A8_ERR_TIMEOUT, zero the workspace again.
+ * Everything else in it is scratch between calls.
  */
 size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
@@ -190,8 +192,10 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
  * capture.  All calls on a device share the one array and leave their
  * scratch in it: calls whose work overlaps on the GPU (different streams
  * without ordering, or other host threads) race and give wrong results, so
- * order them.  What must start at zero is cleared by each call (it always
- * runs the activation kernel and then the decode kernel, one token too).
+ * order them.  What must start at zero starts so (the array is
+ * zero-initialised) and every completed call leaves it so; each call also
+ * runs the activation kernel, which clears the arrival counters, and then
+ * the decode kernel (one token too).
  *   x, packed, y  as for w4a8_linear (device pointers owned by the caller).
  * Limits: M <= 16 (larger M returns W4A8_ERR_SHAPE); any shape needing more
  * scratch than the array holds returns W4A8_ERR_WORKSPACE (no accepted

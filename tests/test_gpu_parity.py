@@ -245,11 +245,13 @@ def test_linear_deterministic_and_workspace_reuse(lib, layer592, m):
     need = max(lib.linear_workspace_bytes(mm, 768, 592) for mm in (1, 5, 16, 300))
     ws = torch.zeros(need + 4096, dtype=torch.uint8, device="cuda")
     a = lib.linear(xt, packed, 592, workspace=ws).clone()
-    # a different shape through the same workspace in between
-    other, _, _ = synth.activations(5, 768, synth.rng_for(8, 99, "act"), 8)
-    lib.linear(bf16(other), packed, 592, workspace=ws)
-    b = lib.linear(xt, packed, 592, workspace=ws)
-    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    # other shapes through the same workspace in between (each path lays out
+    # its scratch differently; the words that must start at zero stay put)
+    for mm in (5, 16, 300, 1):
+        other, _, _ = synth.activations(mm, 768, synth.rng_for(8, 99 + mm, "act"), 8)
+        lib.linear(bf16(other), packed, 592, workspace=ws)
+        b = lib.linear(xt, packed, 592, workspace=ws)
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), mm
 
 
 def test_binding_refuses_bad_arguments(lib, layer592):

@@ -224,9 +224,11 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t ra
 // Tokens are laid out in slices of 16 (the decode kernel runs one launch per
 // slice): token m goes to slice m / 16, `slice_half2` half2 units apart, as
 // token m % 16 of a slice with ceil(tokens in the slice / 8) blocks of 8.
+// The first CTA also clears `zero_count` 16-byte words at `zero_vec` (the
+// decode workspace's split-K counters).
 __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_kernel(
     const uint16_t* __restrict__ x, int M, int K, __half2* __restrict__ out, float* __restrict__ s_x,
-    int slice_half2, unsigned* __restrict__ zero_words, int zero_count) {
+    int slice_half2, uint4* __restrict__ zero_vec, int zero_count) {
   __shared__ float warp_max[kActClusterBlocks];
   __shared__ float cta_max;
   // The previous kernel may still read the workspace: wait before writing.
@@ -235,8 +237,8 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
   const int m = blockIdx.y;
   const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (zero_words && m == 0 && rank == 0) {
-    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_words[i] = 0u;
+  if (zero_vec && m == 0 && rank == 0) {
+    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_vec[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   const int b = int(rank) * kActClusterBlocks + warp;
   const bool mine = b < K / kRotBlock;

@@ -48,6 +48,14 @@ constexpr int kDecWarpsMulti = 12;                 // 2..16 tokens: fewer warps,
 __host__ __device__ constexpr int dec_warps(bool single) { return single ? kDecWarps : kDecWarpsMulti; }
 constexpr int kDecTG = 2;                          // tiles (16 rows each) per unit
 constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
+// The part of a workspace that must hold zeros when a launch starts (every
+// completed launch leaves it so): per CTA boundary, 32 exchange words (a row
+// pair split between two CTAs) and one arrival counter (a pair split among
+// more).  It sits at the workspace's start and has a fixed size, so calls of
+// any shape may share a workspace.
+constexpr size_t kWsXchBytes = size_t(kDecMaxCtas) * 32 * 8;
+constexpr size_t kWsCntOff = kWsXchBytes;
+constexpr size_t kWsZeroBytes = (kWsXchBytes + size_t(kDecMaxCtas) * 4 + 255) / 256 * 256;
 constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
 constexpr int kDecSchRows = 1024;                  // row scales staged in shared memory per CTA
 // Units in flight per warp (register ring depth) per variant.
@@ -64,7 +72,8 @@ struct DecodeParams {
   const float* s_x;      // [M]
   uint16_t* y;           // [M, N] bf16
   float* slots;          // [2 * CTAs][kDecTG * 16][M]: per-CTA partials of pairs shared with other CTAs
-  unsigned* counters;    // [P]
+  unsigned long long* xch;  // [kDecMaxCtas][32]: one token, a pair split between CTAs c and c + 1
+  unsigned* counters;    // [kDecMaxCtas]: arrivals at a pair whose first CTA is c
   unsigned* err;
   int M, N, K, C, T, P, W, U;
   int R, Rm;  // U / W and U % W: warp w's first unit is w R + floor(w Rm / W)
@@ -389,10 +398,16 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 
 // One token: a pair split between warps (levels 2 and 3 of the reduction).
 // Lane l owns row l of the pair (row 16 i + g + 8 h of the partial layout):
-// it adds the contributing warps' partials in warp order, and when the pair
-// also spans other CTAs it parks the CTA's sum in the workspace; the last
-// CTA to arrive (one acquire-release atomic by lane 0) adds the CTAs' sums
-// in CTA order and writes y.
+// it adds the contributing warps' partials in warp order.  A pair that also
+// spans another CTA is finished by whichever of its CTAs comes second:
+//  * two CTAs (the usual case): each lane swaps its CTA's sum, tagged, into
+//    the row's exchange word with one 64-bit atomic; a lane that gets the
+//    other CTA's tagged sum back adds it, writes y and clears the word.  A
+//    sum of two fp32 terms is the same in either order, so the result does
+//    not depend on which CTA arrives first;
+//  * more CTAs: each parks its sum in the workspace and counts itself in with
+//    one acquire-release atomic by lane 0; the last to arrive adds the CTAs'
+//    sums in CTA order and writes y.
 __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, int q0, int q1, int v0, int v1,
                                                const int (&wb)[kDecWarps + 1], uint32_t parts,
                                                uint32_t part_bytes, int lane, const DecEpi& ep) {
@@ -411,28 +426,41 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
     int cf = blockIdx.x, cl = blockIdx.x;
     while (cf > 0 && dec_cta_begin<kDecWarps>(cf, p) > q0) --cf;
     while (dec_cta_begin<kDecWarps>(cl + 1, p) < q1) ++cl;
-    const int sf = dec_slot_floats(1);
-    p.slots[size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf + lane] = tot;
-    __syncwarp();
-    unsigned old = 0;
-    if (lane == 0)
-      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + pr) : "memory");
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != unsigned(cl - cf)) return;  // another CTA finishes this pair
-    __syncwarp();  // the other lanes' loads come after lane 0's acquire
-    tot = 0.f;
-    for (int c0 = cf; c0 <= cl; c0 += 4) {
-      float v[4];
+    if (cl == cf + 1) {
+      unsigned long long* word = p.xch + size_t(cf) * 32 + lane;
+      unsigned long long other;
+      asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;"
+                   : "=l"(other)
+                   : "l"(word), "l"((1ull << 32) | __float_as_uint(tot))
+                   : "memory");
+      if ((other >> 32) == 0) return;  // the other CTA finishes this row
+      *word = 0ull;                    // ready for the next launch on this workspace
+      tot += __uint_as_float(unsigned(other));
+    } else {
+      const int sf = dec_slot_floats(1);
+      p.slots[size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf + lane] = tot;
+      __syncwarp();
+      unsigned old = 0;
+      if (lane == 0)
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + cf) : "memory");
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old != unsigned(cl - cf)) return;  // another CTA finishes this pair
+      __syncwarp();  // the other lanes' loads come after lane 0's acquire
+      tot = 0.f;
+      for (int c0 = cf; c0 <= cl; c0 += 4) {
+        float v[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int cc = c0 + r;
-        const bool have = cc <= cl;
-        v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin<kDecWarps>(cc, p) >= q0 ? 0 : 1)) * sf + lane) : 0.f;
+        for (int r = 0; r < 4; ++r) {
+          const int cc = c0 + r;
+          const bool have = cc <= cl;
+          v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin<kDecWarps>(cc, p) >= q0 ? 0 : 1)) * sf + lane)
+                      : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) tot += v[r];
       }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) tot += v[r];
+      if (lane == 0) p.counters[cf] = 0u;  // ready for the next launch on this workspace
     }
-    if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
   }
   if (row < p.N) {
     const int rr = row - ep.row0;
@@ -893,7 +921,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     __threadfence();
     __syncwarp();
     unsigned old = 0;
-    if (lane == 0) old = atomicAdd(p.counters + pr, 1u);
+    if (lane == 0) old = atomicAdd(p.counters + cf, 1u);
     old = __shfl_sync(0xffffffffu, old, 0);
     if (old != unsigned(cl - cf)) continue;  // another CTA finishes this pair
     __threadfence();
@@ -926,7 +954,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][j][e] += v[r][i][j][e];
     }
-    if (lane == 0) p.counters[pr] = 0u;  // ready for the next launch on this workspace
+    if (lane == 0) p.counters[cf] = 0u;  // ready for the next launch on this workspace
     dec_epilogue<NB>(acc, p, pr, lane, ep);
   }
 }

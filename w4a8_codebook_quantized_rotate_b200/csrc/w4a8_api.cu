@@ -107,7 +107,7 @@ struct LinearPlan {
   int nb;          // decode: token blocks of 8 of a full slice
   int slices;      // decode: launches of up to kDecodeSliceM tokens
   size_t slice_bytes;  // decode: B-fragment bytes of one slice
-  size_t off_sx, off_xq, off_cnt, off_slots, total;
+  size_t off_sx, off_xq, off_slots, total;  // [0, kWsZeroBytes): exchange words and counters
   int T, P, C;
 };
 
@@ -122,18 +122,17 @@ LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
     L.nb = int((mslice + 7) / 8);
     L.slices = int((M + kDecodeSliceM - 1) / kDecodeSliceM);
     L.slice_bytes = size_t(K) * L.nb * 16;
-    L.off_sx = 0;
-    L.off_xq = 256;  // s_x: at most 64 floats
-    L.off_cnt = round_up(L.off_xq + L.slice_bytes * L.slices, 256);
-    L.off_slots = round_up(L.off_cnt + size_t(L.P) * 4, 256);
+    L.off_sx = kWsZeroBytes;
+    L.off_xq = L.off_sx + 256;  // s_x: at most 64 floats
+    L.off_slots = round_up(L.off_xq + L.slice_bytes * L.slices, 256);
     L.total = round_up(L.off_slots + size_t(2) * kDecMaxCtas * dec_slot_floats(int(mslice)) * 4, 256);
   } else {
     L.nb = 0;
     L.slices = 0;
     L.slice_bytes = 0;
-    L.off_sx = 0;
-    L.off_xq = round_up(size_t(M) * 4, 256);
-    L.off_cnt = L.off_slots = 0;
+    L.off_sx = kWsZeroBytes;  // the zero region is left as it is
+    L.off_xq = round_up(L.off_sx + size_t(M) * 4, 256);
+    L.off_slots = 0;
     L.total = round_up(L.off_xq + size_t(M) * K * 2, 256);
   }
   return L;
@@ -294,7 +293,8 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     p.s_x = reinterpret_cast<const float*>(ws + plan.off_sx) + m0;
     p.y = y + m0 * N;
     p.slots = reinterpret_cast<float*>(ws + plan.off_slots);
-    p.counters = reinterpret_cast<unsigned*>(ws + plan.off_cnt);
+    p.xch = reinterpret_cast<unsigned long long*>(ws);
+    p.counters = reinterpret_cast<unsigned*>(ws + kWsCntOff);
     p.err = d->err;
     p.M = int(ms);
     p.N = int(N);
@@ -343,8 +343,8 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
     const unsigned cl = unsigned((K / kRotBlock + kActClusterBlocks - 1) / kActClusterBlocks);
     if (launch_pdl_cluster(rotate_quant_frag_cluster_kernel, dim3(cl, unsigned(M)), dim3(kActClusterThreads), cl, 0,
                            s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x,
-                           int(plan.slice_bytes / 4), reinterpret_cast<unsigned*>(ws + plan.off_cnt),
-                           plan.P) != cudaSuccess)
+                           int(plan.slice_bytes / 4), reinterpret_cast<uint4*>(ws + kWsCntOff),
+                           int((kWsZeroBytes - kWsCntOff) / 16)) != cudaSuccess)
       return W4A8_ERR_CUDA;
   } else {
     if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
@@ -437,9 +437,11 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, c
     }
     scratch = g_static_scratch_ptr[dev];
   }
-  // The split-K counters the decode kernel needs at zero are cleared by the
-  // activation kernel at the start of every call (the two-kernel path, also
-  // for one token); nothing else in the scratch has to start at a known value.
+  // The words the decode kernel needs at zero (exchange words and split-K
+  // counters, at the start of the scratch) are zero in the zero-initialised
+  // array and every completed call leaves them so; the activation kernel of
+  // the two-kernel path (taken here for one token too) also clears the
+  // counters.  Nothing else in the scratch has to start at a known value.
   w4a8_status st = w4a8_linear_prepare(x, M, K, N, scratch, kStaticScratchBytes, stream);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
@@ -541,16 +543,10 @@ w4a8_status w4a8_convert_weight(const float* w, int64_t N, int64_t K, const floa
 
 // ------------------------------------------------------------------ chains of one-token layers
 
-constexpr size_t kChainCounterOff = 256;  // [0, 256): grid-barrier counter
-
-static size_t chain_counter_bytes(const w4a8_chain_layer* layers, int64_t n) {
-  int64_t pmax = 1;
-  for (int64_t i = 0; i < n; ++i) {
-    const int64_t p = (layers[i].N / kTileRows + kDecTG - 1) / kDecTG;
-    pmax = p > pmax ? p : pmax;
-  }
-  return round_up(size_t(pmax) * 4, 256);
-}
+// [0, 256): grid-barrier counter; then the decode zero region (exchange words
+// and split-K counters, shared by the layers); then the per-CTA partials.
+constexpr size_t kChainZeroOff = 256;
+constexpr size_t kChainSlotsOff = kChainZeroOff + kWsZeroBytes;
 
 size_t w4a8_chain_plan_bytes(int64_t n_layers) {
   return n_layers < 1 ? 0 : round_up(size_t(n_layers) * sizeof(DecodeParams), 256);
@@ -560,7 +556,7 @@ size_t w4a8_chain_workspace_bytes(const w4a8_chain_layer* layers, int64_t n_laye
   if (!layers || n_layers < 1) return 0;
   for (int64_t i = 0; i < n_layers; ++i)
     if (!weight_shape_ok(layers[i].N, layers[i].K)) return 0;
-  return kChainCounterOff + chain_counter_bytes(layers, n_layers) +
+  return kChainSlotsOff +
          round_up(size_t(2) * kDecMaxCtas * dec_slot_floats(1) * 4, 256);
 }
 
@@ -581,8 +577,9 @@ w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, vo
   DeviceState* d = nullptr;
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  unsigned* counters = reinterpret_cast<unsigned*>(ws + kChainCounterOff);
-  float* slots = reinterpret_cast<float*>(ws + kChainCounterOff + chain_counter_bytes(layers, n_layers));
+  unsigned long long* xch = reinterpret_cast<unsigned long long*>(ws + kChainZeroOff);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + kChainZeroOff + kWsCntOff);
+  float* slots = reinterpret_cast<float*>(ws + kChainSlotsOff);
   const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
   DecodeParams* host = new (std::nothrow) DecodeParams[size_t(n_layers)];
   if (!host) return W4A8_ERR_SHAPE;
@@ -599,6 +596,7 @@ w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, vo
     p.s_x = nullptr;
     p.y = L.y;
     p.slots = slots;
+    p.xch = xch;
     p.counters = counters;
     p.err = d->err;
     p.M = 1;
@@ -624,13 +622,12 @@ w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace, 
                            void* stream) {
   if (!plan || !workspace) return W4A8_ERR_NULL;
   if (n_layers < 1 || n_layers > (int64_t(1) << 20)) return W4A8_ERR_SHAPE;
-  if (workspace_bytes < kChainCounterOff + 256) return W4A8_ERR_WORKSPACE;
+  if (workspace_bytes < kChainSlotsOff) return W4A8_ERR_WORKSPACE;
   DeviceState* d = nullptr;
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the barrier and the split-K counters start at zero
-  const size_t zero = workspace_bytes < kChainCounterOff + (size_t(1) << 16) ? workspace_bytes
-                                                                              : kChainCounterOff + (size_t(1) << 16);
+  const size_t zero = kChainSlotsOff;
   if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return W4A8_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas));
