@@ -58,12 +58,17 @@ __device__ __forceinline__ void fwht8_in_lane(float (&v)[8]) {
   }
 }
 
-// Lane's 8 values of the rotated 256-block b of a bf16 row: positions
-// 256 b + 8 lane .. + 7.  Three butterfly stages inside the lane, five across
-// lanes (shuffles), then the exact 1/16.
-__device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ row, int b, int lane, float (&v)[8]) {
-  // L2 only: a chain of layers rewrites its activation buffers within one launch
-  const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8));
+// The lane's 16 bytes of 256-block b of a bf16 row (positions 256 b + 8 lane
+// .. + 7), from L2 only: a chain of layers rewrites its activation buffers
+// within one launch.
+__device__ __forceinline__ uint4 load_block_lane(const uint16_t* __restrict__ row, int b, int lane) {
+  return __ldcg(reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8));
+}
+
+// Lane's 8 values of a rotated 256-block, from the lane's 16 bytes of it.
+// Three butterfly stages inside the lane, five across lanes (shuffles), then
+// the exact 1/16.
+__device__ __forceinline__ void rotate_words_lane(const uint4 raw, int lane, float (&v)[8]) {
   const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -82,6 +87,11 @@ __device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ r
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;  // 1/16, exact
+}
+
+// Lane's 8 values of the rotated 256-block b of a bf16 row.
+__device__ __forceinline__ void rotate_block_lane(const uint16_t* __restrict__ row, int b, int lane, float (&v)[8]) {
+  rotate_words_lane(load_block_lane(row, b, lane), lane, v);
 }
 
 // Per-token scale and code: s = amax / 127 (IEEE division), q = clamp(rint(v / s), -127, 127)

@@ -396,8 +396,8 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 }
 
-// One token: a pair split between warps (levels 2 and 3 of the reduction).
-// Lane l owns row l of the pair (row 16 i + g + 8 h of the partial layout):
+// One token: a pair split between warps (levels 2 and 3 of the reduction);
+// CTAs cf..cl hold parts of it.  Lane l owns row l of the pair (row 16 i + g + 8 h of the partial layout):
 // it adds the contributing warps' partials in warp order.  A pair that also
 // spans another CTA is finished by whichever of its CTAs comes second:
 //  * two CTAs (the usual case): each lane swaps its CTA's sum, tagged, into
@@ -409,7 +409,7 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 //    one acquire-release atomic by lane 0; the last to arrive adds the CTAs'
 //    sums in CTA order and writes y.
 __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, int q0, int q1, int v0, int v1,
-                                               const int (&wb)[kDecWarps + 1], uint32_t parts,
+                                               int cf, int cl, const int (&wb)[kDecWarps + 1], uint32_t parts,
                                                uint32_t part_bytes, int lane, const DecEpi& ep) {
   float tot = 0.f;
 #pragma unroll
@@ -423,9 +423,6 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
   const int row = pr * (kDecTG * 16) + lane;
   if (!(q0 >= v0 && q1 <= v1)) {
     // level 3: the pair spans CTAs cf..cl
-    int cf = blockIdx.x, cl = blockIdx.x;
-    while (cf > 0 && dec_cta_begin<kDecWarps>(cf, p) > q0) --cf;
-    while (dec_cta_begin<kDecWarps>(cl + 1, p) < q1) ++cl;
     if (cl == cf + 1) {
       unsigned long long* word = p.xch + size_t(cf) * 32 + lane;
       unsigned long long other;
@@ -500,6 +497,7 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
 // of layers with it; `wait_inputs` is where the body waits for what an
 // earlier step wrote (the activations, and the workspace it reuses).
 struct DecWaitPdl {
+  static constexpr int kLoadsAhead = 4;  // kept blocks whose loads are all issued before the first transform
   __device__ __forceinline__ void operator()() const { pdl_wait(); }
 };
 
@@ -516,7 +514,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
   const uint32_t sch_s = parts + uint32_t(kW * 2) * part_bytes;  // row scales
   const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
-  const uint32_t wbeg_s = sx_s + 64;                                      // warp range starts [17]
+  const uint32_t wbeg_s = sx_s + 64;  // warp range starts [17]; at +96 the CTA pair context [4]
   const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int cta_w0 = blockIdx.x * kW;
@@ -558,6 +556,17 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(wl) * 4u), "r"(u0));
     if (wl == kW - 1) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wbeg_s + uint32_t(kW) * 4u), "r"(v1));
   }
+  // The CTA's first and last pairs and the CTAs where those start and end,
+  // for the reduction after the loop (worked out now, while the previous
+  // grid runs, so that the tail has no divisions).
+  const uint32_t ctx_s = wbeg_s + 96u;
+  if (threadIdx.x == kThr - 1 && v1 > v0) {
+    const int plo = v0 / p.C, phi = (v1 - 1) / p.C;
+    int cf = blockIdx.x, cl = blockIdx.x;
+    while (cf > 0 && dec_cta_begin<kW>(cf, p) > plo * p.C) --cf;
+    while (dec_cta_begin<kW>(cl + 1, p) < (phi + 1) * p.C) ++cl;
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ctx_s), "r"(plo), "r"(phi), "r"(cf), "r"(cl));
+  }
   DecEpi ep;
   ep.sch = sch_s;
   ep.sx = sx_s;
@@ -594,11 +603,20 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     constexpr int kKeep = 4;
     float amax = 0.f;
     float vk[kKeep][8];
+    // the first kLoadsAhead kept blocks' loads are in flight before the first transform
+    constexpr int kAhead = Wait::kLoadsAhead < kKeep ? Wait::kLoadsAhead : kKeep;
+    uint4 raw[kAhead];
+#pragma unroll
+    for (int jj = 0; jj < kAhead; ++jj) {
+      const int j = wl + kW * jj;
+      if (j < nown) raw[jj] = load_block_lane(p.x, int(crank) + int(ncta) * j, lane);
+    }
 #pragma unroll
     for (int jj = 0; jj < kKeep; ++jj) {
       const int j = wl + kW * jj;
       if (j < nown) {
-        rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, vk[jj]);
+        rotate_words_lane(jj < kAhead ? raw[jj] : load_block_lane(p.x, int(crank) + int(ncta) * j, lane), lane,
+                          vk[jj]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(vk[jj][i]));
       }
@@ -871,15 +889,22 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 #pragma unroll
   for (int i = 0; i <= kW; ++i)
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wb[i]) : "r"(wbeg_s + uint32_t(i) * 4u));
-  const int pair_lo = v0 / p.C, pair_hi = (v1 - 1) / p.C;
+  int pair_lo, pair_hi, cta_first, cta_last;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(pair_lo), "=r"(pair_hi), "=r"(cta_first), "=r"(cta_last)
+               : "r"(ctx_s));
   for (int pr = pair_lo + wl; pr <= pair_hi; pr += kW) {
     const int q0 = pr * p.C, q1 = q0 + p.C;  // the pair's units [q0, q1)
     bool whole = false;                       // one warp held all of it (and wrote y)
 #pragma unroll
     for (int ww = 0; ww < kW; ++ww) whole |= (wb[ww] <= q0) & (wb[ww + 1] >= q1);
     if (whole) continue;
+    // CTAs cf..cl hold parts of the pair: only the CTA's first pair starts
+    // before it and only its last one ends after it
+    const int cf = pr == pair_lo ? cta_first : int(blockIdx.x);
+    const int cl = pr == pair_hi ? cta_last : int(blockIdx.x);
     if constexpr (SINGLE) {
-      dec_reduce_one(p, pr, q0, q1, v0, v1, wb, parts, part_bytes, lane, ep);
+      dec_reduce_one(p, pr, q0, q1, v0, v1, cf, cl, wb, parts, part_bytes, lane, ep);
       continue;
     }
     // the contributors' partials, added in warp order (all loads independent)
@@ -903,9 +928,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       continue;
     }
     // ---- level 3: the pair spans CTAs cf..cl; park this CTA's partial in the workspace
-    int cf = blockIdx.x, cl = blockIdx.x;
-    while (cf > 0 && dec_cta_begin<kW>(cf, p) > q0) --cf;
-    while (dec_cta_begin<kW>(cl + 1, p) < q1) ++cl;
     const int sf = dec_slot_floats(p.M);
     const int g = lane >> 2, t = lane & 3;
     float* mine = p.slots + size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf;
@@ -976,6 +998,7 @@ __global__ void __launch_bounds__(dec_warps(SINGLE) * 32, 1) decode_kernel(const
 // nothing in the chain writes them.  The barrier counter is bounded: a
 // CTA that waits about a second records a timeout and goes on.
 struct DecWaitChain {
+  static constexpr int kLoadsAhead = 1;  // (registers: the chain keeps more state live)
   unsigned* ctr;    // arrivals: CTAs add 1 after each layer
   unsigned target;  // arrivals that mean the previous layer is complete (0: the first layer)
   unsigned* err;
