@@ -531,6 +531,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8 +
                       (SINGLE ? 4 * (lane & 1) : 0);
 
+  // The codebook level this lane puts in the table: loaded ahead of the
+  // weight stream so that it does not queue behind it.
+  const float level = p.cb[lane & 15];
+
   DecStage<NB, SINGLE> st[D];
   // Weights do not depend on the previous kernel: start streaming them first.
   // (x for more than one token comes from it, so it is loaded after the wait.)
@@ -571,21 +575,23 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   ep.sch = sch_s;
   ep.sx = sx_s;
   ep.row0 = (v0 / p.C) * (kDecTG * 16);
-  {
-    const int rows = min(kDecSchRows, min(p.N, (v1 > v0 ? (v1 - 1) / p.C + 1 : 0) * kDecTG * 16) - ep.row0);
-    for (int i = threadIdx.x; i < rows; i += kThr)
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(sch_s + uint32_t(i) * 4u), "f"(__ldg(p.sch + ep.row0 + i)));
+  // The CTA's row scales: loaded now, written to shared memory just before
+  // the barrier that ends the activation step (no wait for them here).
+  const int sch_rows = min(kDecSchRows, min(p.N, (v1 > v0 ? (v1 - 1) / p.C + 1 : 0) * kDecTG * 16) - ep.row0);
+  constexpr int kSchPer = (kDecSchRows + kThr - 1) / kThr;
+  float sch_r[kSchPer];
+#pragma unroll
+  for (int j = 0; j < kSchPer; ++j) {
+    const int i = int(threadIdx.x) + j * kThr;
+    sch_r[j] = i < sch_rows ? __ldg(p.sch + ep.row0 + i) : 0.f;
   }
   // Table: entry b for lane l at lut + 256 b + 4 l holds fp16 (cb[b & 15], cb[b >> 4]).
-  {
-    const float level = p.cb[lane & 15];
-    for (int b = wl; b < 256; b += kW) {
-      const float lo = __shfl_sync(0xffffffffu, level, b & 15);
-      const float hi = __shfl_sync(0xffffffffu, level, b >> 4);
-      const __half2 h = __floats2half2_rn(lo, hi);
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(lane) * 4u),
-                   "r"(*reinterpret_cast<const uint32_t*>(&h)));
-    }
+  for (int b = wl; b < 256; b += kW) {
+    const float lo = __shfl_sync(0xffffffffu, level, b & 15);
+    const float hi = __shfl_sync(0xffffffffu, level, b >> 4);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(lut + (uint32_t(b) << 8) + uint32_t(lane) * 4u),
+                 "r"(*reinterpret_cast<const uint32_t*>(&h)));
   }
   wait_inputs();  // activations, scales and counters come from an earlier step
   int cx = first_c;  // chunk of the next x fragment to load (more than one token)
@@ -701,6 +707,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
         }
       }
     }
+  }
+#pragma unroll
+  for (int j = 0; j < kSchPer; ++j) {
+    const int i = int(threadIdx.x) + j * kThr;
+    if (i < sch_rows) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sch_s + uint32_t(i) * 4u), "f"(sch_r[j]));
   }
   __syncthreads();
 
