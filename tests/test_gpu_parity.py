@@ -334,6 +334,36 @@ def test_one_token_small_grids_and_long_pairs(lib, n, k):
     check_linear(y_one.float().cpu().numpy(), O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
 
 
+# The words at the start of every workspace that join partial sums across
+# CTAs: per CTA boundary (148) 32 eight-byte exchange words and one 4-byte
+# arrival counter, rounded up to 256 bytes.
+ZERO_REGION_BYTES = (148 * 32 * 8 + 148 * 4 + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 5120, 17408), (1, 17408, 5120), (1, 8448, 16), (4, 17408, 5120),
+                                   (16, 5120, 4096), (40, 768, 592), (300, 768, 592)])
+def test_workspace_zero_region_left_at_zero(lib, m, k, n):
+    """Every completed call, whatever its path (one-token kernel, two-kernel
+    path, 2-16-token decode, slices, GEMM), leaves the exchange words and
+    arrival counters at zero, which is what the next call on the workspace
+    needs; and a region filled with garbage by nothing else stays so."""
+    q = synth.quantized_format_device(n, k, seed=5, device="cuda")
+    packed = lib.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"])
+    bits, _, _ = synth.activations(m, k, synth.rng_for(17, m + k, "act"), max(1, k // 100))
+    xt = bf16(bits)
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    assert ws.numel() > ZERO_REGION_BYTES
+    y = lib.linear(xt, packed, n, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:ZERO_REGION_BYTES].count_nonzero()) == 0
+    if m <= 64:
+        lib.linear_prepare(xt, n, ws)
+        y_run = lib.linear_run(m, k, packed, n, ws)
+        torch.cuda.synchronize()
+        assert int(ws[:ZERO_REGION_BYTES].count_nonzero()) == 0
+        assert torch.equal(y.view(torch.int16), y_run.view(torch.int16))
+
+
 @pytest.mark.parametrize("m", [1, 3, 20, 80])
 def test_linear_zero_token_and_zero_rows(lib, m):
     """An all-zero token gives s_x = 0 and a zero output row; an all-zero
