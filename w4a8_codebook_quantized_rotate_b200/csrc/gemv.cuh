@@ -617,6 +617,16 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       const int j = wl + kW * jj;
       if (j < nown) raw[jj] = load_block_lane(p.x, int(crank) + int(ncta) * j, lane);
     }
+    // The warp's next 8 units (after the 4 in its register ring) into L2 with
+    // one bulk prefetch, issued behind the token's loads: the memory system
+    // streams them while the CTA rotates and quantises the token.
+    {
+      const int pa = min(u0 + D, u1), pb = min(u0 + 3 * D, u1);
+      if (lane == 0 && pb > pa)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.units + size_t(pa) * kUnitBytes),
+                     "r"(uint32_t(pb - pa) * uint32_t(kUnitBytes))
+                     : "memory");
+    }
 #pragma unroll
     for (int jj = 0; jj < kKeep; ++jj) {
       const int j = wl + kW * jj;
