@@ -29,10 +29,12 @@
 // consecutive ranges.  A warp that covers a whole tile pair writes y
 // directly.  A pair split between warps is reduced in two levels, both in a
 // fixed order (the result is deterministic): the warps of a CTA leave their
-// partials in shared memory and one warp adds them after a CTA barrier; a
-// pair that also crosses into another CTA leaves one partial per CTA in the
-// workspace, and the last CTA to finish it (an atomic counter, no waiting)
-// adds those and writes y.
+// partials in shared memory and one warp adds them after a CTA barrier.  A
+// pair that also crosses into one other CTA (one token) is joined through
+// one 64-bit exchange word per row, and the second CTA to arrive adds the
+// two sums (two fp32 terms: the same in either order); otherwise each CTA
+// leaves its partial in the workspace and the last to finish (an atomic
+// counter, no waiting) adds them in CTA order and writes y.
 #pragma once
 
 #include <type_traits>
@@ -480,9 +482,9 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
 // directly.  A pair split between warps is reduced in two levels, both in a
 // fixed order (the result is deterministic): the warps of a CTA leave their
 // partials in shared memory and one warp adds them after a CTA barrier; a
-// pair that also crosses into another CTA leaves one partial per CTA in the
-// workspace, and the last CTA to finish it (an atomic counter, no waiting)
-// adds those and writes y.
+// pair that also crosses into other CTAs is finished by the CTA that comes
+// last to it (dec_reduce_one for one token, the counter path below for
+// more).
 //
 // FUSED (one token): the kernel also does the activation step: every CTA
 // rotates the bf16 row and quantises it to int8 (the activation kernel's
