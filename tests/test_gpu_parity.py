@@ -221,10 +221,13 @@ def test_linear_exact_integer_case(lib, m):
 
 
 @pytest.mark.parametrize("m,k,n", [(1, 5120, 17408), (1, 17408, 5120), (4, 17408, 5120), (16, 17408, 5120),
+                                   (1, 5120, 10240), (1, 5120, 5120), (64, 17408, 5120), (128, 17408, 5120),
                                    (4096, 5120, 17408), (8192, 17408, 5120)])
 def test_linear_full_size_sampled(lib, m, k, n):
-    """Workload shapes in the launch configuration the benchmark times; the
-    oracle computes a sample of outputs (tokens x output rows)."""
+    """Workload shapes in the launch configuration the benchmark times (the
+    decode step's four projections at one token, the down projection at 1,
+    4, 16, 64 and 128 tokens, both prefill shapes); the oracle computes a
+    sample of outputs (tokens x output rows)."""
     q = synth.quantized_format(n, k, synth.rng_for(11, n, "qfmt"))
     bits, x, _ = synth.activations(m, k, synth.rng_for(11, m, "act"), max(1, k // 100))
     y = lib.linear(bf16(bits), pack(lib, q), n)
