@@ -60,11 +60,22 @@ def test_bad_weight_shapes_have_zero_size(lib, n, k):
     assert lib.w4a8_linear_workspace_bytes(1, k, n) == 0
 
 
+# Every workspace starts with the words that join partial sums across CTAs:
+# per CTA boundary (148) 32 eight-byte exchange words and a 4-byte counter.
+ZERO_REGION_BYTES = (148 * 32 * 8 + 148 * 4 + 255) // 256 * 256
+
+
 def test_workspace_sizes(lib):
     assert lib.w4a8_linear_workspace_bytes(0, 256, 16) == 0
     dec = lib.w4a8_linear_workspace_bytes(1, 5120, 17408)
     pre = lib.w4a8_linear_workspace_bytes(4096, 5120, 17408)
     assert dec > 5120 * 16 and pre >= 4096 * 5120 * 2 + 4096 * 4
+    # the region is there for every shape, ahead of the activations (and, for
+    # the GEMM, of s_x and the fp16 x_q)
+    assert dec >= ZERO_REGION_BYTES + 256 + 5120 * 16
+    assert pre >= ZERO_REGION_BYTES + 4096 * 4 + 4096 * 5120 * 2
+    for m in (1, 2, 9, 16, 17, 64, 65, 300):
+        assert lib.w4a8_linear_workspace_bytes(m, 768, 592) > ZERO_REGION_BYTES
 
 
 def test_null_and_shape_errors_before_launch(lib):
