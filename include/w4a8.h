@@ -324,6 +324,17 @@ w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const 
  */
 w4a8_status w4a8_get_device_error(void* stream);
 
+/*
+ * Self-test of the device error path (the pages have no counterpart): one
+ * small kernel runs the library's two kinds of bounded wait, an mbarrier
+ * phase and a global word, on things that never complete, so both give up
+ * after a short bound (about a millisecond at most) and record a timeout.
+ * The next w4a8_get_device_error on the stream then returns
+ * W4A8_ERR_TIMEOUT and clears the word; the context stays usable.  Nothing
+ * traps or hangs.  Errors: ARCH, CUDA.
+ */
+w4a8_status w4a8_selftest_timeout(void* stream);
+
 /* Static English description of a status code. */
 const char* w4a8_status_string(w4a8_status status);
 

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
         "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_prepare",
         "w4a8_linear_run",
         "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
-        "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_status_string", "w4a8_unpack_dequant"])
+        "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_selftest_timeout", "w4a8_status_string",
+        "w4a8_unpack_dequant"])
 
 
 def test_library_exports_every_declared_symbol(lib):

@@ -272,6 +272,22 @@ def test_no_device_error_recorded(lib):
     assert lib.get_device_error() == 0
 
 
+def test_bounded_waits_report_a_timeout_and_the_context_stays_usable(lib, layer592):
+    """The library's bounded device waits (an mbarrier phase, a global word),
+    run on things that never complete, give up, record a timeout that the
+    next get_device_error returns and clears; the layer still runs and
+    matches the oracle afterwards."""
+    c, packed, wmax = layer592
+    assert lib.get_device_error() == 0
+    lib.selftest_timeout()
+    assert lib.get_device_error() == 6  # W4A8_ERR_TIMEOUT
+    assert lib.get_device_error() == 0  # cleared
+    bits, x, _ = synth.activations(3, 768, synth.rng_for(19, 3, "act"), 8)
+    y = lib.linear(bf16(bits), packed, 592).float().cpu().numpy()
+    assert lib.get_device_error() == 0
+    check_linear(y, O.linear(x, c["idx"], c["s_rel"], c["s_ch"], c["cb"]), x, wmax)
+
+
 @pytest.mark.parametrize("m", [1, 4, 300])
 def test_prepare_once_run_several_layers(lib, m):
     """One prepared activation, several layers of the same shape, each run

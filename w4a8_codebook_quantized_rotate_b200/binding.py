@@ -24,7 +24,7 @@ STATUS = {
 EXPORTS = (
     "w4a8_packed_bytes", "w4a8_pack_layout", "w4a8_unpack_dequant", "w4a8_rotate_quant_act",
     "w4a8_linear_workspace_bytes", "w4a8_linear", "w4a8_linear_prepare", "w4a8_linear_run",
-    "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_status_string",
+    "w4a8_linear_decode_static", "w4a8_get_device_error", "w4a8_selftest_timeout", "w4a8_status_string",
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
     "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
@@ -65,6 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_linear_run": (st, [i64, i64, vp, i64, vp, vp, sz, vp]),
         "w4a8_linear_decode_static": (st, [vp, i64, i64, vp, i64, vp, vp]),
         "w4a8_get_device_error": (st, [vp]),
+        "w4a8_selftest_timeout": (st, [vp]),
         "w4a8_status_string": (ctypes.c_char_p, [st]),
         "w4a8_convert_workspace_bytes": (sz, [i64, i64, i64]),
         "w4a8_convert_weight": (st, [vp, i64, i64, vp, vp, i64, ctypes.c_int32, ctypes.c_double,
@@ -226,6 +227,12 @@ def linear_decode_static(x: torch.Tensor, packed: torch.Tensor, n: int, out: tor
 def get_device_error(stream=None) -> int:
     """Synchronise and return (and clear) the device error status (0 = ok)."""
     return int(load_library().w4a8_get_device_error(_stream(stream)))
+
+
+def selftest_timeout(stream=None) -> None:
+    """Run the device self-test of the bounded waits (they record a timeout
+    that the next get_device_error returns)."""
+    _check("w4a8_selftest_timeout", load_library().w4a8_selftest_timeout(_stream(stream)))
 
 
 def convert_weight(w: torch.Tensor, codebook: torch.Tensor | None = None, sample_pos: torch.Tensor | None = None,

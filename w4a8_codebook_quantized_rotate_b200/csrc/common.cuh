@@ -168,6 +168,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Bounded poll of a global word until it reaches `target` (acquire loads,
+// one L2 round trip each).  Returns false (and records a timeout in the
+// error word) if it did not within `max_tries` polls.
+__device__ __forceinline__ bool poll_at_least_bounded(const unsigned* word, unsigned target, unsigned* err,
+                                                      uint32_t max_tries) {
+  for (uint32_t i = 0; i < max_tries; ++i) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
+    if (v >= target) return true;
+  }
+  record_error(err, kErrTimeout);
+  return false;
+}
+
 // ---------------------------------------------------------------- TMA (no multicast)
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {

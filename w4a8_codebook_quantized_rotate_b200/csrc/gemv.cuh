@@ -1030,15 +1030,7 @@ struct DecWaitChain {
       pdl_wait();
       return;
     }
-    if (threadIdx.x == 0) {
-      bool done = false;
-      for (uint32_t i = 0; i < (1u << 26) && !done; ++i) {  // an L2 round trip per poll: about a second
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        done = v >= target;
-      }
-      if (!done) record_error(err, kErrTimeout);
-    }
+    if (threadIdx.x == 0) poll_at_least_bounded(ctr, target, err, 1u << 26);  // about a second
     __syncthreads();
   }
 };

@@ -193,6 +193,26 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 }
 
 }  // namespace
+
+// A word nothing ever writes: the self-test's flag.
+__device__ unsigned g_never_set;
+
+// The library's two kinds of bounded device wait, each on something that
+// never completes: an mbarrier phase nobody arrives at (the GEMM's role
+// handshakes) and a global word nobody sets (the chain's grid barrier).
+// Each gives up after `tries` polls and records a timeout.
+__global__ void wait_timeout_selftest_kernel(unsigned* err, uint32_t tries) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_wait_bounded(&bar, 0, err, tries);
+    poll_at_least_bounded(&g_never_set, 1u, err, tries);
+  }
+}
 }  // namespace w4a8
 
 using namespace w4a8;
@@ -674,6 +694,13 @@ w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const 
   if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   dense_reference_kernel<<<unsigned((N + kRefWarps - 1) / kRefWarps), kRefWarps * 32, 0,
                            static_cast<cudaStream_t>(stream)>>>(x, M, K, w, N, y);
+  return launch_status();
+}
+
+w4a8_status w4a8_selftest_timeout(void* stream) {
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(d->err, 1024u);
   return launch_status();
 }
 
