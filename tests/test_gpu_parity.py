@@ -383,6 +383,38 @@ def test_workspace_zero_region_left_at_zero(lib, m, k, n):
         assert torch.equal(y.view(torch.int16), y_run.view(torch.int16))
 
 
+GUARD = 64  # elements of guard band on each side of an output (keeps 16-byte alignment)
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 768, 592), (1, 8448, 16), (1, 17408, 272), (5, 768, 592), (16, 256, 16),
+                                   (40, 768, 592), (300, 768, 592)])
+def test_outputs_leave_guard_bands_untouched(lib, m, k, n):
+    """y written into the middle of a larger buffer filled with a canary
+    pattern: every path writes exactly its [M, N] outputs (the canaries on
+    both sides survive) and the same bits as into a buffer of its own; the
+    same for the standalone dequant's fp32 output."""
+    q = synth.quantized_format_device(n, k, seed=9, device="cuda")
+    packed = lib.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"])
+    bits, _, _ = synth.activations(m, k, synth.rng_for(21, m + k, "act"), max(1, k // 100))
+    xt = bf16(bits)
+    canary = 0x7BAD
+    buf = torch.full((m * n + 2 * GUARD,), canary, dtype=torch.int16, device="cuda")
+    y = buf[GUARD:GUARD + m * n].view(torch.bfloat16).view(m, n)
+    lib.linear(xt, packed, n, out=y)
+    ref = lib.linear(xt, packed, n)
+    torch.cuda.synchronize()
+    assert bool((buf[:GUARD] == canary).all()) and bool((buf[GUARD + m * n:] == canary).all())
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    if m == 1:
+        dbuf = torch.full((n * k + 2 * GUARD,), -7.25, dtype=torch.float32, device="cuda")
+        st = lib.load_library().w4a8_unpack_dequant(packed.data_ptr(), n, k, dbuf[GUARD:].data_ptr(),
+                                                    torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert bool((dbuf[:GUARD] == -7.25).all()) and bool((dbuf[GUARD + n * k:] == -7.25).all())
+        assert torch.equal(dbuf[GUARD:GUARD + n * k].view(n, k), lib.unpack_dequant(packed, n, k))
+
+
 @pytest.mark.parametrize("m", [1, 3, 20, 80])
 def test_linear_zero_token_and_zero_rows(lib, m):
     """An all-zero token gives s_x = 0 and a zero output row; an all-zero
