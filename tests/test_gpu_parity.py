@@ -383,6 +383,28 @@ def test_workspace_zero_region_left_at_zero(lib, m, k, n):
         assert torch.equal(y.view(torch.int16), y_run.view(torch.int16))
 
 
+def test_one_workspace_shared_by_layers_of_different_shapes(lib):
+    """A decode step shares one workspace among layers of different (K, N)
+    (and token counts): each call gives the same bits as with a fresh
+    workspace of its own, in any order, twice over."""
+    shapes = [(768, 592), (8448, 16), (17408, 272), (5120, 2048), (256, 4096)]
+    layers, xs, fresh = [], [], []
+    for i, (k, n) in enumerate(shapes):
+        q = synth.quantized_format_device(n, k, seed=30 + i, device="cuda")
+        layers.append(lib.pack_layout(q["packed"], q["s_rel"], q["s_ch"], q["cb"]))
+        m = 1 if i % 2 == 0 else 3
+        bits, _, _ = synth.activations(m, k, synth.rng_for(23, i, "act"), max(1, k // 100))
+        xs.append(bf16(bits))
+        fresh.append(lib.linear(xs[-1], layers[-1], n).clone())
+    need = max(lib.linear_workspace_bytes(x.shape[0], k, n) for x, (k, n) in zip(xs, shapes))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for order in (range(len(shapes)), reversed(range(len(shapes))), [0, 2, 4, 1, 3]):
+        for i in order:
+            k, n = shapes[i]
+            y = lib.linear(xs[i], layers[i], n, workspace=ws)
+            assert torch.equal(y.view(torch.int16), fresh[i].view(torch.int16)), shapes[i]
+
+
 GUARD = 64  # elements of guard band on each side of an output (keeps 16-byte alignment)
 
 
