@@ -174,35 +174,57 @@ def oracle_sample(rows: int):
     import synth
     q = synth.quantized_format(N_DEC, K_DEC, synth.rng_for(1, 0, "qfmt"))
     bits, x, _ = synth.activations(M_DEC, K_DEC, synth.rng_for(1, 0, "act"), K_DEC // 100)
-    return q, x
+    return q, bits, x
 
 
 def time_oracle(q, x, rows: int, reps: int):
     """Oracle linear on ``rows`` output rows, ``reps`` times, one BLAS thread.
-    Returns (seconds per rep, weight bytes per rep)."""
+    Returns (seconds per rep, weight bytes per rep, the last rep's output)."""
     import oracle as O
     from threadpoolctl import threadpool_limits
     sel = np.arange(rows)
+    y = None
     with threadpool_limits(limits=1):
         O.linear_packed(x, q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=sel[: min(rows, 64)])  # warm
         t0 = time.perf_counter()
         for _ in range(reps):
-            O.linear_packed(x, q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=sel)
+            y = O.linear_packed(x, q["packed"], q["s_rel"], q["s_ch"], q["cb"], rows=sel)
         dt = (time.perf_counter() - t0) / reps
-    return dt, weight_bytes(rows, K_DEC)
+    return dt, weight_bytes(rows, K_DEC), y
 
 
-def cpu_baseline(budget_s: float = 15.0) -> dict:
-    q, x = oracle_sample(N_DEC)
-    dt1, _ = time_oracle(q, x, 1024, 1)
+def cpu_baseline(budget_s: float = 15.0, B=None, torch=None, dev=None) -> dict:
+    """The oracle timed on a bounded row sample of the C1 layer.  With the
+    library at hand (B), the same layer also runs through w4a8_linear on the
+    GPU and the sampled rows are compared with the oracle's (relative L2,
+    and the largest per-row error over the bar 1e-2 * ||x|| * max|W_hat|)."""
+    q, bits, x = oracle_sample(N_DEC)
+    dt1, _, _ = time_oracle(q, x, 1024, 1)
     rows = int(min(N_DEC, max(256, 1024 * (budget_s / 3) / max(dt1, 1e-6))))
     rows -= rows % 16
     reps = max(1, int(budget_s / max(dt1 * rows / 1024, 1e-6)))
     reps = min(reps, 5)
-    dt, nbytes = time_oracle(q, x, rows, reps)
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"oracle linear (rotate+quantise x, three-tier dequant, fp64 matmul) on {rows} of "
-                      f"{N_DEC} output rows of the M=1 K=5120 layer, {reps} repeats, 1 thread"}
+    dt, nbytes, y_ref = time_oracle(q, x, rows, reps)
+    out = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"oracle linear (rotate+quantise x, three-tier dequant, fp64 matmul) on {rows} of "
+                     f"{N_DEC} output rows of the M=1 K=5120 layer, {reps} repeats, 1 thread"}
+    if B is not None:
+        import oracle as O
+        t = {kk: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for kk, v in q.items()}
+        packed = B.pack_layout(t["packed"], t["s_rel"], t["s_ch"], t["cb"])
+        xt = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = B.linear(xt, packed, N_DEC)[:, :rows].double().cpu().numpy()
+        err = y - y_ref
+        wmax = float(np.abs(O.dequant_packed(q["packed"], q["s_rel"], q["s_ch"], q["cb"],
+                                             rows=np.arange(rows))).max())
+        bar = 1e-2 * np.linalg.norm(np.asarray(x, dtype=np.float64), axis=1) * wmax
+        out["parity"] = {"rows": rows,
+                         "rel_l2": float(np.linalg.norm(err) / np.linalg.norm(y_ref)),
+                         "max_abs_over_bar": float((np.abs(err).max(axis=1) / bar).max()),
+                         "how": "the same seeded layer and token through w4a8_linear on the GPU (one "
+                                "kernel), its first rows against the oracle's; bars: rel_l2 <= 2e-3, "
+                                "max_abs_over_bar <= 1"}
+    return out
 
 
 def max_over_ranks(v: float, world: int, device) -> float:
@@ -227,9 +249,9 @@ def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    q, x = oracle_sample(N_DEC)
+    q, _, x = oracle_sample(N_DEC)
     # size each step so that warmup + steps take about two minutes in all
-    dt1, _ = time_oracle(q, x, 256, 1)
+    dt1, _, _ = time_oracle(q, x, 256, 1)
     per_row = dt1 / 256
     rows = int(max(16, min(N_DEC, (args.ref_seconds / max(1, args.steps + args.warmup)) / per_row)))
     rows -= rows % 16
@@ -866,7 +888,7 @@ def main() -> None:
         "device_error": err,
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline"] = cpu_baseline(B=B, torch=torch, dev=dev)
     print(json.dumps(line), flush=True)
 
 
