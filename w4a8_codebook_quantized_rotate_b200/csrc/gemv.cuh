@@ -538,8 +538,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const float level = p.cb[lane & 15];
 
   DecStage<NB, SINGLE> st[D];
-  // Weights do not depend on the previous kernel: start streaming them first.
-  // (x for more than one token comes from it, so it is loaded after the wait.)
+  // Weights do not depend on the previous kernel: start streaming them now,
+  // before the wait.  (x for more than one token comes from it, so it is
+  // loaded after the wait.)
   if constexpr (SINGLE) {
     // one token: slot d holds the next unit u with u % D == d (see the loop below)
 #pragma unroll
