@@ -1,0 +1,45 @@
+"""Host-side pieces of the benchmark that need no GPU: the algorithmic byte
+count of a layer, and the rule that a committed DRAM-traffic figure is only
+reported while the kernel source it was captured from is unchanged."""
+
+from __future__ import annotations
+
+import json
+import os
+
+import pytest
+
+import bench
+
+
+def test_weight_bytes_is_the_packed_layer():
+    # 0.5 B of index and 1/16 B of group scale per weight, 4 B per row, 64 B of codebook
+    assert bench.weight_bytes(17408, 5120) == 17408 * 5120 // 2 + 17408 * 5120 // 16 + 4 * 17408 + 64
+    assert bench.weight_bytes(17408, 5120) == 50204736
+
+
+def test_committed_traffic_matches_its_source_hash():
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    files = {"decode_kernel_fused": ["gemv.cuh", "act.cuh", "common.cuh"],
+             "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"]}
+    for kernel, srcs in files.items():
+        got = bench.profiled_traffic(kernel, srcs)
+        if d[kernel]["source_sha256_16"] == bench.kernel_source_hash(srcs):
+            assert got == pytest.approx(d[kernel]["dram_bytes_per_launch"])
+            # both captures are of launches that read the whole 50.2 MB layer at least once
+            assert got >= bench.weight_bytes(17408, 5120)
+        else:
+            assert got is None
+
+
+def test_traffic_is_withheld_when_the_source_changes(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k": {"source_sha256_16": "0" * 16, "dram_bytes_per_launch": 123}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "1" * 16)
+    assert bench.profiled_traffic("k", ["x"]) is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "0" * 16)
+    assert bench.profiled_traffic("k", ["x"]) == 123
+    assert bench.profiled_traffic("missing", ["x"]) is None
