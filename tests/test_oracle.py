@@ -162,6 +162,41 @@ def test_lloyd_fixed_point_conditions():
     assert np.all(np.diff(lv) > 0)
 
 
+def test_lloyd_residuals_hand_computed_non_fixed_point():
+    # Worked by hand.  Two levels (-1, 3): the midpoint is 1, and the sample
+    # value 1 sits on it, so it belongs to the lower cell.  Lower cell
+    # {-3, -2, -1, 1}: mean -5/4, residual |-1 - (-5/4)| = 1/4.  Upper cell
+    # {2, 4}: mean 3, residual 0.  (Had the tie gone up, the lower cell's mean
+    # would be -2 and the residual 1.)
+    s = np.array([4.0, -1.0, 2.0, -3.0, 1.0, -2.0])   # unsorted on purpose
+    worst, empty = O.lloyd_residuals(s, np.array([-1.0, 3.0]))
+    assert worst == 0.25 and empty == 0
+    # A sign error (level + mean) or a cell taken on the wrong side of the
+    # midpoint would show here: upper level 2 against a cell mean of 3.
+    worst, empty = O.lloyd_residuals(s, np.array([-1.0, 2.0]))
+    # midpoint 0.5: lower {-3, -2, -1} mean -2 -> 1; upper {1, 2, 4} mean 7/3 -> 1/3
+    assert worst == 1.0 and empty == 0
+
+
+def test_lloyd_residuals_hand_computed_empty_cell():
+    # Three levels (0.5, 2, 5): midpoints 1.25 and 3.5.  Cells {0, 0.25, 0.5}
+    # (mean 0.25, residual 0.25), {} (empty), {5, 5.5, 6} (mean 5.5,
+    # residual 0.5).  All values are exact in binary.
+    s = np.array([0.0, 0.25, 0.5, 5.0, 5.5, 6.0])
+    worst, empty = O.lloyd_residuals(s, np.array([0.5, 2.0, 5.0]))
+    assert worst == 0.5 and empty == 1
+    # the same sample at its own fixed point: levels = cell means, one cell empty
+    worst, empty = O.lloyd_residuals(s, np.array([0.25, 2.0, 5.5]))
+    assert worst == 0.0 and empty == 1
+    # The fit starts at the 1/6, 1/2, 5/6 quantiles (linear interpolation:
+    # 5/24, 11/4, 67/12); the middle cell (1.479.., 4.166..] is empty, so one
+    # round gives (1/4, 11/4, 11/2) with the empty cell's level kept, and
+    # that is a fixed point with one empty cell.
+    lv, rounds = O.lloyd_max(s, 3, max_iter=1, tol=0.0)
+    assert rounds == 1 and np.array_equal(lv, [0.25, 2.75, 5.5])
+    assert O.lloyd_residuals(s, lv) == (0.0, 1)
+
+
 def test_lloyd_empty_cell_keeps_level():
     # two far clusters and 16 levels: quantile init puts levels inside the
     # clusters, so no cell is empty -- but a sample of identical values leaves
