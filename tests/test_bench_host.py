@@ -43,3 +43,25 @@ def test_traffic_is_withheld_when_the_source_changes(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "0" * 16)
     assert bench.profiled_traffic("k", ["x"]) == 123
     assert bench.profiled_traffic("missing", ["x"]) is None
+
+
+def test_source_hash_ignores_comments_only():
+    a = "int f(int x) {\n  return x + 1;  // one more\n}\n"
+    b = "/* a block\n   comment */\nint f(int x) {\n\n  return x + 1;\n}  // trailing\n"
+    c = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench.strip_comments(a) == bench.strip_comments(b)
+    assert bench.strip_comments(a) != bench.strip_comments(c)
+
+
+def test_oracle_pool_splits_rows_over_processes():
+    import numpy as np
+    import synth
+    q = synth.quantized_format(64, 256, synth.rng_for(9, 0, "qfmt"))
+    _, x, _ = synth.activations(1, 256, synth.rng_for(9, 0, "act"), 2)
+    pool = bench.OraclePool(q, x)
+    try:
+        assert 1 <= pool.workers <= bench.OraclePool.MAX_WORKERS
+        assert pool.run(48) > 0.0
+    finally:
+        pool.close()
+    assert np.isfinite(bench.weight_bytes(48, 256))
