@@ -184,25 +184,26 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
  * allocator of its own.
  *
  * Instead of a workspace it uses a scratch array built into the library: a
- * file-scope __device__ array of W4A8_STATIC_SCRATCH_BYTES (16 MiB), which
- * every GPU that loads the library holds until the process exits.  The call
+ * file-scope __device__ array of W4A8_STATIC_SCRATCH_BYTES (2 MiB; the
+ * largest plan, M = 16 at K = W4A8_MAX_K, needs about 1.62 MiB), which every
+ * GPU that loads the library holds until the process exits.  The call
  * allocates nothing and calls no allocating routine.  Its first call on a
  * device looks up the array's device address once (cudaGetSymbolAddress,
- * with that device current); make that first call before any stream
- * capture.  All calls on a device share the one array and leave their
- * scratch in it: calls whose work overlaps on the GPU (different streams
- * without ordering, or other host threads) race and give wrong results, so
- * order them.  What must start at zero starts so (the array is
- * zero-initialised) and every completed call leaves it so; each call also
- * runs the activation kernel, which clears the arrival counters, and then
- * the decode kernel (one token too).
+ * with that device current, after the architecture check); make that first
+ * call before any stream capture.  All calls on a device share the one
+ * array and leave their scratch in it: calls whose work overlaps on the GPU
+ * (different streams without ordering, or other host threads) race and give
+ * wrong results, so order them.  Each call runs the activation kernel, which
+ * clears the words the decode kernel needs at zero (exchange words and
+ * arrival counters), and then the decode kernel (one token too); so a call
+ * that reported W4A8_ERR_TIMEOUT needs no reset before the next one.
  *   x, packed, y  as for w4a8_linear (device pointers owned by the caller).
- * Limits: M <= 16 (larger M returns W4A8_ERR_SHAPE); any shape needing more
- * scratch than the array holds returns W4A8_ERR_WORKSPACE (no accepted
+ * Limits: M <= 16 (larger M returns W4A8_ERR_SHAPE); a shape needing more
+ * scratch than the array holds would return W4A8_ERR_WORKSPACE (no accepted
  * (N, K) does at M <= 16).
  * Errors: NULL, SHAPE, WORKSPACE, ALIGN, ARCH, CUDA.
  */
-#define W4A8_STATIC_SCRATCH_BYTES (16u << 20)
+#define W4A8_STATIC_SCRATCH_BYTES (2u << 20)
 w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K,
                                       const void* packed, int64_t N, uint16_t* y,
                                       void* stream);

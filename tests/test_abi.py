@@ -121,3 +121,15 @@ def test_convert_refuses_bad_arguments_without_a_gpu(lib):
     # null pointers and shapes are checked before any device work
     assert lib.w4a8_convert_weight(None, 16, 256, None, None, 0, 500, 1e-12, None, None, None, None, None,
                                    None, 0, None) == 1
+
+
+def test_static_scratch_holds_every_decode_plan(lib):
+    # The built-in scratch of w4a8_linear_decode_static must hold the
+    # workspace of every shape it accepts (M <= 16, any N, K up to the
+    # maximum), and should not be much larger than the largest of them.
+    size = int(re.search(r"#define W4A8_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(HEADER).read())
+               .group(1)) << 20
+    need = max(lib.w4a8_linear_workspace_bytes(m, k, n)
+               for m in (1, 2, 8, 9, 16) for k in (256, 8192, 8448, 32768) for n in (16, 5120, 17408, 1 << 20))
+    assert 0 < need <= size
+    assert size <= 2 * need

@@ -348,8 +348,11 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
   return W4A8_OK;
 }
 
-w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+// The activation step before w4a8_linear_run.  `zero_from` is where the
+// activation kernel starts clearing the workspace's zero region (the split-K
+// counters by default; the static-scratch call clears it whole).
+static w4a8_status prepare_impl(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
+                                size_t workspace_bytes, void* stream, size_t zero_from) {
   if (!x) return W4A8_ERR_NULL;
   if (!aligned16(x)) return W4A8_ERR_ALIGN;
   LinearPlan plan;
@@ -363,8 +366,8 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
     const unsigned cl = unsigned((K / kRotBlock + kActClusterBlocks - 1) / kActClusterBlocks);
     if (launch_pdl_cluster(rotate_quant_frag_cluster_kernel, dim3(cl, unsigned(M)), dim3(kActClusterThreads), cl, 0,
                            s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x,
-                           int(plan.slice_bytes / 4), reinterpret_cast<uint4*>(ws + kWsCntOff),
-                           int((kWsZeroBytes - kWsCntOff) / 16)) != cudaSuccess)
+                           int(plan.slice_bytes / 4), reinterpret_cast<uint4*>(ws + zero_from),
+                           int((kWsZeroBytes - zero_from) / 16)) != cudaSuccess)
       return W4A8_ERR_CUDA;
   } else {
     if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
@@ -372,6 +375,11 @@ w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t
       return W4A8_ERR_CUDA;
   }
   return launch_status();
+}
+
+w4a8_status w4a8_linear_prepare(const uint16_t* x, int64_t M, int64_t K, int64_t N, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return prepare_impl(x, M, K, N, workspace, workspace_bytes, stream, kWsCntOff);
 }
 
 w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N, uint16_t* y, void* workspace,
@@ -440,11 +448,19 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* pac
 static void* g_static_scratch_ptr[kMaxDevices];
 static std::mutex g_static_scratch_mutex;
 
+// The largest scratch a call may need: M = 16 at the largest K (the plan
+// does not depend on N).  The array's size is checked against it once, and
+// a CPU test checks the header's constant against w4a8_linear_workspace_bytes.
+static_assert(kStaticScratchBytes % 256 == 0, "the scratch size is a whole number of 256-byte blocks");
+
 w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, const void* packed, int64_t N,
                                       uint16_t* y, void* stream) {
   if (!x || !packed || !y) return W4A8_ERR_NULL;
   if (M > kDecodeSliceM || !act_shape_ok(M, K) || !weight_shape_ok(N, K)) return W4A8_ERR_SHAPE;
   if (linear_plan(M, K, N).total > kStaticScratchBytes) return W4A8_ERR_WORKSPACE;
+  // architecture first: on another GPU the array's lookup would fail with no kernel image
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
   void* scratch = nullptr;
@@ -452,17 +468,20 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, c
     std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
     if (!g_static_scratch_ptr[dev]) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return W4A8_ERR_CUDA;
+      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();  // leave no error behind for a later launch check
+        return W4A8_ERR_CUDA;
+      }
       g_static_scratch_ptr[dev] = p;
     }
     scratch = g_static_scratch_ptr[dev];
   }
-  // The words the decode kernel needs at zero (exchange words and split-K
-  // counters, at the start of the scratch) are zero in the zero-initialised
-  // array and every completed call leaves them so; the activation kernel of
-  // the two-kernel path (taken here for one token too) also clears the
-  // counters.  Nothing else in the scratch has to start at a known value.
-  w4a8_status st = w4a8_linear_prepare(x, M, K, N, scratch, kStaticScratchBytes, stream);
+  // Every call clears the whole zero region (exchange words and split-K
+  // counters, at the start of the scratch) in its activation kernel before
+  // the decode kernel runs, so a call cut short (a timeout) leaves nothing
+  // that a later call could trip on.  Nothing else in the scratch has to
+  // start at a known value.
+  w4a8_status st = prepare_impl(x, M, K, N, scratch, kStaticScratchBytes, stream, 0);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
 }
