@@ -532,6 +532,20 @@ def measure_c3(B, synth, torch, dev, rank, stream, steps, warmup):
                  (wu, 17408, 5120, out_o.reshape(-1), up_o.reshape(-1)),
                  (wd, 5120, 17408, up_o.reshape(-1), h.reshape(-1))]
         xin = h.reshape(-1)
+    # the same step with each layer quantising the next layer's activation (one launch per layer)
+    fused = B.DecodeChain(desc)
+    for i in range(warmup):
+        fused.run()
+    replay = graph_loop(lambda i: fused.run(), steps, stream, chunk=4)
+    replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_fused = e0.elapsed_time(e1) / steps
+    same_fused = bool(torch.equal(h.view(torch.int16), y_calls.view(torch.int16)))
+    del replay, fused
     plan, cws, nl = B.chain_plan(desc)
     for i in range(warmup):
         B.chain_run(plan, nl, cws)
@@ -552,6 +566,11 @@ def measure_c3(B, synth, torch, dev, rank, stream, steps, warmup):
             "ms_per_step": ms_calls, "weight_GBs": total / (ms_calls * 1e-3) / 1e9, "weight_bytes_per_step": total,
             "resident_bytes": resident, "kernels_per_step": C3_BLOCKS * len(C3_SHAPES), "steps": steps,
             "how": "310 w4a8_linear calls, one kernel each, replayed from CUDA graphs",
+            "decode_chain": {"ms_per_step": ms_fused, "weight_GBs": total / (ms_fused * 1e-3) / 1e9,
+                             "kernels_per_step": C3_BLOCKS * len(C3_SHAPES),
+                             "how": "w4a8_decode_chain: one launch per layer; each layer rotates the next layer's "
+                                    "input blocks in its epilogue and the next layer only quantises them",
+                             "same_bits_as_layer_by_layer": same_fused},
             "persistent_chain": {"ms_per_step": ms, "weight_GBs": total / (ms * 1e-3) / 1e9, "kernels_per_step": 1,
                                  "how": "one persistent launch of the 310 layers (w4a8_chain_run), grid barrier "
                                         "between layers",

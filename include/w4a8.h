@@ -141,10 +141,13 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   y          output [M, N] bf16 bit patterns (uint16), row-major.
  *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
  * M <= 64 runs the decode kernel (a weight-streaming GEMV, one launch per
- * slice of up to 16 tokens); larger M runs the tensor-core GEMM.  For one token a single kernel rotates, quantises
- * and applies the layer (every CTA quantises the token itself, with the
- * activation kernel's arithmetic); otherwise the call is
- * w4a8_linear_prepare followed by w4a8_linear_run.  Two calls sharing one
+ * slice of up to 16 tokens); larger M runs the tensor-core GEMM, except that
+ * 64 <= M <= 256 on a layer of fewer than 100 row tiles of 128 (where the
+ * GEMM would leave most SMs idle) runs a small-batch tensor-core kernel
+ * that splits the weight stream over every SM.  For one token a single
+ * kernel rotates, quantises and applies the layer (every CTA quantises the
+ * token itself, with the activation kernel's arithmetic); otherwise the call
+ * is w4a8_linear_prepare followed by w4a8_linear_run.  Two calls sharing one
  * workspace must be ordered on the GPU (same stream, or synchronised).
  * Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA.
  */
@@ -247,6 +250,34 @@ w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, vo
                             void* stream);
 w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * A decode step as one launch per one-token layer, each layer quantising the
+ * next layer's activation in its own epilogue (ConvRot card, "Why this
+ * exists": a decode step re-reads every layer's weights for one token, so
+ * the per-layer work besides that stream must shrink).  The layers are the
+ * chain descriptors above.  A layer whose input x lies inside an earlier
+ * layer's output y (at a multiple of 256 elements, wholly inside, and
+ * written by no layer in between) reads that output already rotated: the
+ * producing layer rotates each 256-block of the consumer's input as soon as
+ * all its rows are written (the last writer of the block does it) and keeps
+ * the running absmax, so the consumer only quantises (same arithmetic, so
+ * the same codes and s_x as w4a8_linear on the same bf16 x).  Other layers
+ * rotate their x themselves.  Results equal the layer-by-layer w4a8_linear
+ * calls bit for bit; y buffers are written as those calls would.
+ *   layers     host array of n_layers descriptors (as for w4a8_chain_plan),
+ *              run strictly in order.
+ *   workspace  device, w4a8_decode_chain_workspace_bytes(layers, n) bytes,
+ *              zero-filled before its first use (like a w4a8_linear
+ *              workspace: its first 38,656 bytes must be zero when a call
+ *              starts, and every completed call leaves them so).
+ * The call issues one small memset and one kernel launch per layer on
+ * `stream` (capturable in a CUDA graph).  Two calls sharing a workspace must
+ * be ordered.  Errors: NULL, SHAPE, ALIGN, WORKSPACE, ARCH, CUDA.
+ */
+size_t w4a8_decode_chain_workspace_bytes(const w4a8_chain_layer* layers, int64_t n_layers);
+w4a8_status w4a8_decode_chain(const w4a8_chain_layer* layers, int64_t n_layers, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /*
  * Weight converter on the GPU: fp32 W [N, K] -> the four stored tensors

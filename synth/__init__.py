@@ -99,3 +99,43 @@ def quantized_format_device(n: int, k: int, seed: int, device):
     s_ch = torch.rand(n, generator=g, device=device, dtype=torch.float32) * 0.1 + 0.05
     cb = torch.from_numpy(codebook(np.random.Generator(np.random.PCG64(seed)))).to(device)
     return {"packed": packed, "s_rel": s_rel, "s_ch": s_ch, "cb": cb}
+
+
+EXTREME_CODEBOOK = np.array([-8.0, -4.5, -2.5, -1.5, -0.9, -0.5, -0.2, -3e-5, 2e-5, 0.15, 0.4, 0.8, 1.3,
+                             2.2, 4.0, 7.5], dtype=np.float32)
+
+
+def quantized_format_edges(n: int, k: int, rng: np.random.Generator) -> dict:
+    """Stored-format tensors at the edges of the format: group-scale codes
+    mixed with e4m3 subnormals (codes 1..7) and zeros inside live rows, a row
+    with every group scale zero, a row whose only live group is its first,
+    a row with a zero row scale, and a codebook with two levels within 1e-4
+    of zero and levels out to -8 and 7.5.  Indices uniform over all bytes."""
+    if n < 4:
+        raise ValueError("needs at least 4 rows")
+    s_rel = rng.integers(32, 57, size=(n, k // 16), dtype=np.uint8)
+    u = rng.random(size=s_rel.shape)
+    s_rel[u < 0.15] = rng.integers(1, 8, size=int((u < 0.15).sum()), dtype=np.uint8)   # subnormal codes
+    s_rel[(u >= 0.15) & (u < 0.22)] = 0                                                # zero groups
+    s_rel[0] = 0                                  # a dead row
+    s_rel[1, 1:] = 0                              # one live group
+    s_ch = rng.uniform(0.05, 0.15, size=n).astype(np.float32)
+    s_ch[2] = 0.0                                 # a zero row scale
+    return {"packed": rng.integers(0, 256, size=(n, k // 2), dtype=np.uint8), "s_rel": s_rel,
+            "s_ch": s_ch, "cb": EXTREME_CODEBOOK.copy()}
+
+
+def weights_with_edges(n: int, k: int, rng: np.random.Generator) -> np.ndarray:
+    """:func:`weights` with edge rows for the converter: an all-zero row, a
+    row with one large entry (300, about 10^4 times the rest: its other
+    groups' ratios to the row maximum fall to e4m3 subnormals or zero), a
+    row whose first half is zero, and a row with one zero block of 256 (16
+    zero groups, after rotation too) between live ones."""
+    if n < 5 or k < 768:
+        raise ValueError("needs at least 5 rows and 768 columns")
+    w = weights(n, k, rng)
+    w[1] = 0.0
+    w[2, 5] = 300.0
+    w[3, : k // 2] = 0.0
+    w[4, 256:512] = 0.0
+    return w

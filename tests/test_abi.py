@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "w4a8_chain_plan", "w4a8_chain_plan_bytes", "w4a8_chain_run", "w4a8_chain_workspace_bytes",
         "w4a8_compare", "w4a8_compare_workspace_bytes", "w4a8_convert_weight", "w4a8_convert_workspace_bytes",
-        "w4a8_dense_reference",
+        "w4a8_decode_chain", "w4a8_decode_chain_workspace_bytes", "w4a8_dense_reference",
         "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_prepare",
         "w4a8_linear_run",
         "w4a8_linear_workspace_bytes", "w4a8_pack_layout",

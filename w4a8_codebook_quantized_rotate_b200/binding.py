@@ -28,6 +28,7 @@ EXPORTS = (
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
     "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
+    "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain",
 )
 
 
@@ -77,6 +78,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_chain_workspace_bytes": (sz, [vp, i64]),
         "w4a8_chain_plan": (st, [vp, i64, vp, sz, vp, sz, vp]),
         "w4a8_chain_run": (st, [vp, i64, vp, sz, vp]),
+        "w4a8_decode_chain_workspace_bytes": (sz, [vp, i64]),
+        "w4a8_decode_chain": (st, [vp, i64, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -386,3 +389,31 @@ def chain_run(plan: torch.Tensor, n_layers: int, workspace: torch.Tensor, stream
     lib = load_library()
     _check("w4a8_chain_run", lib.w4a8_chain_run(plan.data_ptr(), n_layers, workspace.data_ptr(), workspace.numel(),
                                                 _stream(stream)))
+
+
+class DecodeChain:
+    """A decode step as one launch per one-token layer, each layer quantising
+    the next one's activation (w4a8_decode_chain).  ``layers`` as for
+    :func:`chain_plan`; the tensors must outlive the runs."""
+
+    def __init__(self, layers):
+        lib = load_library()
+        self._arr = (ChainLayer * len(layers))()
+        dev = None
+        for i, (packed, n, k, x, y) in enumerate(layers):
+            _cuda(packed, torch.uint8, "packed")
+            _cuda(x, torch.bfloat16, "x")
+            _cuda(y, torch.bfloat16, "y")
+            if x.numel() != k or y.numel() != n:
+                raise ValueError(f"layer {i}: x must hold K and y N values")
+            self._arr[i] = ChainLayer(packed.data_ptr(), n, k, x.data_ptr(), y.data_ptr())
+            dev = packed.device
+        self.n_layers = len(layers)
+        need = lib.w4a8_decode_chain_workspace_bytes(self._arr, self.n_layers)
+        if need == 0:
+            raise W4A8Error("w4a8_decode_chain_workspace_bytes", 2)
+        self.workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+
+    def run(self, stream=None) -> None:
+        _check("w4a8_decode_chain", load_library().w4a8_decode_chain(
+            self._arr, self.n_layers, self.workspace.data_ptr(), self.workspace.numel(), _stream(stream)))

@@ -84,7 +84,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
 // of a second before the kernel records a timeout and unwinds.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, TcShared* sh, unsigned* err) {
   for (uint32_t i = 0; i < (1u << 20); ++i) {
+#if W4A8_SPIN_WAIT
+    if (mbar_test_wait(bar, parity)) return true;
+#else
     if (mbar_try_wait(bar, parity)) return true;
+#endif
     if ((i & 1023u) == 1023u && sh->abort) return false;
   }
   sh->abort = 1;

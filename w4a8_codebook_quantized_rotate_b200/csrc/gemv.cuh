@@ -79,6 +79,26 @@ struct DecodeParams {
   unsigned* err;
   int M, N, K, C, T, P, W, U;
   int R, Rm;  // U / W and U % W: warp w's first unit is w R + floor(w Rm / W)
+  // one token (gemv1.cuh): the P C / 2 duos are split over G CTAs, CTA c
+  // holding [c Dq + min(c, Dr), (c + 1) Dq + min(c + 1, Dr))
+  int G, Dq, Dr;
+  // One token in a decode chain (gemv1.cuh), all optional (null: unused):
+  //  * producer: outputs [act_off, act_off + act_len) are the next layer's
+  //    input; each 256-block of them, once all its rows are written, is
+  //    rotated into act_rot (fp32) and its absmax folded into *act_amax
+  //    (float bits, an atomic maximum); act_cnt counts written rows per block;
+  //  * consumer: the token's rotated values and absmax come from the
+  //    previous producer (in_rot, in_amax) instead of x;
+  //  * zero_cnt[0 .. zero_n): cleared after the wait (the counters and absmax
+  //    word of the set the next producer writes).
+  float* act_rot;
+  unsigned* act_cnt;
+  unsigned* act_amax;
+  int act_off, act_len;
+  const float* in_rot;
+  const unsigned* in_amax;
+  unsigned* zero_cnt;
+  int zero_n;
 };
 
 // Floats of one partial (a tile pair, the first M tokens).
@@ -1011,44 +1031,6 @@ __global__ void __launch_bounds__(dec_warps(SINGLE) * 32, 1) decode_kernel(const
   // this grid's completion before it touches anything this grid writes.
   pdl_launch_dependents();
   decode_body<NB, D, SINGLE, FUSED>(p, DecWaitPdl{});
-}
-
-// ---------------------------------------------------------------------------
-// A chain of one-token layers in one persistent launch (a decode step: each
-// layer's input is an earlier layer's output).  Every CTA runs every layer
-// with the fused body; between layers a grid barrier (all CTAs co-resident:
-// cooperative launch) makes the previous layer's y visible.  A layer's
-// weights, table and row scales are fetched before the barrier, since
-// nothing in the chain writes them.  The barrier counter is bounded: a
-// CTA that waits about a second records a timeout and goes on.
-struct DecWaitChain {
-  static constexpr int kLoadsAhead = 1;  // (registers: the chain keeps more state live)
-  unsigned* ctr;    // arrivals: CTAs add 1 after each layer
-  unsigned target;  // arrivals that mean the previous layer is complete (0: the first layer)
-  unsigned* err;
-  __device__ __forceinline__ void operator()() const {
-    if (target == 0) {  // the first layer waits for the previous kernel
-      pdl_wait();
-      return;
-    }
-    if (threadIdx.x == 0) poll_at_least_bounded(ctr, target, err, 1u << 26);  // about a second
-    __syncthreads();
-  }
-};
-
-__global__ void __launch_bounds__(kDecThreads, 1)
-    decode_chain_kernel(const DecodeParams* __restrict__ layers, int n_layers, unsigned* barrier) {
-  pdl_launch_dependents();
-#pragma unroll 1
-  for (int l = 0; l < n_layers; ++l) {
-    const DecodeParams p = layers[l];  // a local copy: the body keeps what it uses in registers
-    decode_body<1, kDecDepthSingle, true, true>(p, DecWaitChain{barrier, unsigned(l) * gridDim.x, p.err});
-    __syncthreads();  // this CTA is done with layer l (its y and workspace writes issued)
-    if (threadIdx.x == 0) {
-      __threadfence();
-      atomicAdd(barrier, 1u);
-    }
-  }
 }
 
 }  // namespace w4a8

@@ -3,14 +3,17 @@
 // ownership and error behaviour, are in include/w4a8.h.
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "w4a8.h"
 
 #include "act.cuh"
 #include "common.cuh"
 #include "convert.cuh"
+#include "gemm_sk.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv1.cuh"
 #include "pack.cuh"
 #include "verify.cuh"
 
@@ -77,12 +80,13 @@ w4a8_status device_state(DeviceState** out) {
       d.err = static_cast<unsigned*>(sym);
       if (allow_smem(rotate_quant_kernel<kActI8Row>, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(rotate_quant_kernel<kActF16Row>, size_t(kMaxK) * 4) != cudaSuccess ||
-          allow_smem(decode_kernel<1, kDecDepthSingle, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
-          allow_smem(decode_kernel<1, kDecDepthSingle, true, true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
+          allow_smem(decode_one_kernel<false>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
+          allow_smem(decode_one_kernel<true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_chain_kernel, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
           allow_smem(decode_kernel<2, kDecDepth2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
-          allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess)
+          allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess ||
+          allow_smem(gemm_sk_kernel, 232448) != cudaSuccess)  // the largest sk_smem_bytes over token tiles
         return W4A8_ERR_CUDA;
     }
     d.ready = true;
@@ -96,14 +100,26 @@ w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK
 
 // ------------------------------------------------------------------ linear workspace
 
-// Up to 64 tokens run the decode kernel, in slices of up to 16 tokens (one
-// launch per slice; the weights stream once per slice).  Past that the
-// tensor-core GEMM is faster.
+// One token runs the one-token decode kernel, 2..64 tokens the mma.sync
+// decode kernel in slices of up to 16 tokens, more the prefill GEMM -- except
+// that 64..256 tokens on a layer with few 128-row tiles (the GEMM would leave
+// most SMs idle: 40 CTAs at N = 5120) run the small-batch tensor-core kernel,
+// which splits the weight stream over every SM.
 constexpr int kDecodeSliceM = 16;
 constexpr int kDecodeMaxM = 64;
+#ifndef W4A8_SK_MIN_M
+#define W4A8_SK_MIN_M 64
+#endif
+constexpr int64_t kSkMinM = W4A8_SK_MIN_M;
+constexpr int64_t kSkMaxRowTiles = 100;  // more 128-row tiles than this keep the GEMM busy enough
+
+static_assert(size_t(kSkMaxCtas) * 8 * 4 <= kWsXchBytes, "the small-batch counters fit in the zero region");
 
 struct LinearPlan {
   bool decode;
+  bool sk;         // the small-batch tensor-core kernel
+  int nt;          // sk: token tile (M rounded up to 16)
+  size_t off_part; // sk: partial tiles
   int nb;          // decode: token blocks of 8 of a full slice
   int slices;      // decode: launches of up to kDecodeSliceM tokens
   size_t slice_bytes;  // decode: B-fragment bytes of one slice
@@ -111,9 +127,10 @@ struct LinearPlan {
   int T, P, C;
 };
 
-LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
+LinearPlan linear_plan(int64_t M, int64_t K, int64_t N, bool allow_sk = true) {
   LinearPlan L{};
-  L.decode = M <= kDecodeMaxM;
+  L.sk = allow_sk && M >= kSkMinM && M <= kSkMaxTokens && (N + kSkRows - 1) / kSkRows < kSkMaxRowTiles;
+  L.decode = !L.sk && M <= kDecodeMaxM;
   L.T = int(N / kTileRows);
   L.C = int(K / kChunkK);
   L.P = (L.T + kDecTG - 1) / kDecTG;
@@ -134,6 +151,11 @@ LinearPlan linear_plan(int64_t M, int64_t K, int64_t N) {
     L.off_xq = round_up(L.off_sx + size_t(M) * 4, 256);
     L.off_slots = 0;
     L.total = round_up(L.off_xq + size_t(M) * K * 2, 256);
+    if (L.sk) {
+      L.nt = int((M + 15) / 16 * 16);
+      L.off_part = L.total;  // [CTAs][2][nt][128] fp32
+      L.total = round_up(L.off_part + size_t(kSkMaxCtas) * 2 * L.nt * kSkRows * 4, 256);
+    }
   }
   return L;
 }
@@ -295,6 +317,14 @@ static w4a8_status linear_checks(int64_t M, int64_t K, int64_t N, const void* wo
 #endif
 constexpr int64_t kDecPairK = W4A8_DEC_PAIR_K;
 
+// One-token work split (gemv1.cuh): the P C / 2 duos over G CTAs.
+static void one_token_split(DecodeParams& p, int ctas_avail) {
+  const int duos = p.P * p.C / 2;
+  p.G = duos < ctas_avail ? duos : ctas_avail;
+  p.Dq = duos / p.G;
+  p.Dr = duos % p.G;
+}
+
 // Decode launch (M <= 16).  With x given (one token) the kernel also rotates
 // and quantises the token; otherwise it reads what w4a8_linear_prepare left
 // in the workspace.
@@ -304,7 +334,7 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
   for (int sl = 0; sl < plan.slices; ++sl) {
     const int64_t m0 = int64_t(sl) * kDecodeSliceM;
     const int64_t ms = M - m0 < kDecodeSliceM ? M - m0 : kDecodeSliceM;
-    DecodeParams p;
+    DecodeParams p{};  // the decode-chain fields stay null
     p.x = x;
     p.units = pk + L.off_units;
     p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
@@ -324,21 +354,22 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     p.P = plan.P;
     p.U = plan.P * plan.C;
     const int wpc = dec_warps(ms == 1);  // warps per CTA of this variant
-    const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * wpc;
+    const int ctas_avail = d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas;
+    const int warps_avail = ctas_avail * wpc;
     p.W = p.U < warps_avail ? p.U : warps_avail;
     p.R = p.U / p.W;
     p.Rm = p.U % p.W;
-    const dim3 grid((p.W + wpc - 1) / wpc);
+    one_token_split(p, ctas_avail);
+    const dim3 grid(ms == 1 ? unsigned(p.G) : unsigned((p.W + wpc - 1) / wpc));
     const size_t smem = dec_smem_bytes(int(ms), int(K), ms == 1);
     const int nb = int((ms + 7) / 8);
     cudaError_t e;
     if (x && K > kDecPairK)  // pairs of CTAs share the activation step (an even grid; extra CTAs hold no units)
-      e = launch_pdl_cluster(decode_kernel<1, kDecDepthSingle, true, true>, dim3((grid.x + 1) & ~1u),
-                             dim3(kDecThreads), 2, smem, s, p);
+      e = launch_pdl_cluster(decode_one_kernel<true>, dim3((grid.x + 1) & ~1u), dim3(kOneThreads), 2, smem, s, p);
     else if (x)
-      e = launch_pdl(decode_kernel<1, kDecDepthSingle, true, true>, grid, dim3(kDecThreads), smem, s, p);
+      e = launch_pdl(decode_one_kernel<true>, grid, dim3(kOneThreads), smem, s, p);
     else if (ms == 1)
-      e = launch_pdl(decode_kernel<1, kDecDepthSingle, true>, grid, dim3(kDecThreads), smem, s, p);
+      e = launch_pdl(decode_one_kernel<false>, grid, dim3(kOneThreads), smem, s, p);
     else if (nb == 1)
       e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(wpc * 32), smem, s, p);
     else
@@ -403,12 +434,38 @@ w4a8_status w4a8_linear_run(int64_t M, int64_t K, const void* packed, int64_t N,
   CUtensorMap tmap;
   const cuuint64_t gdim[2] = {cuuint64_t(K), cuuint64_t(M)};
   const cuuint64_t gstride[1] = {cuuint64_t(K) * 2};
-  const cuuint32_t box[2] = {uint32_t(kTcBK), uint32_t(kTcTokens)};
+  const cuuint32_t box[2] = {uint32_t(kTcBK), uint32_t(plan.sk ? plan.nt : kTcTokens)};
   const cuuint32_t estride[2] = {1, 1};
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xq, gdim, gstride, box, estride,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return W4A8_ERR_CUDA;
+  if (plan.sk) {
+    SkParams q;
+    q.units = pk + L.off_units;
+    q.sch = reinterpret_cast<const float*>(pk + L.off_sch);
+    q.cb = reinterpret_cast<const float*>(pk + L.off_cb);
+    q.s_x = s_x;
+    q.y = y;
+    q.part = reinterpret_cast<float*>(ws + plan.off_part);
+    q.counters = reinterpret_cast<unsigned*>(ws);  // inside the zero region (the exchange words' place)
+    q.err = d->err;
+    q.M = int(M);
+    q.N = int(N);
+    q.K = int(K);
+    q.C = plan.C;
+    q.RT = int((N + kSkRows - 1) / kSkRows);
+    q.NT = plan.nt;
+    const int items = q.RT * q.C;
+    const int ctas = d->sms < kSkMaxCtas ? d->sms : kSkMaxCtas;
+    q.G = items < ctas ? items : ctas;
+    q.Iq = items / q.G;
+    q.Ir = items % q.G;
+    q.idesc = (1u << 4) | (uint32_t(q.NT >> 3) << 17) | (uint32_t(kSkRows >> 4) << 24);
+    const cudaError_t e =
+        launch_pdl(gemm_sk_kernel, dim3(unsigned(q.G)), dim3(kSkThreads), sk_smem_bytes(q.NT), s, tmap, q);
+    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+  }
   TcParams p;
   p.units = pk + L.off_units;
   p.sch = reinterpret_cast<const float*>(pk + L.off_sch);
@@ -476,11 +533,14 @@ w4a8_status w4a8_linear_decode_static(const uint16_t* x, int64_t M, int64_t K, c
     }
     scratch = g_static_scratch_ptr[dev];
   }
-  // Every call clears the whole zero region (exchange words and split-K
-  // counters, at the start of the scratch) in its activation kernel before
-  // the decode kernel runs, so a call cut short (a timeout) leaves nothing
-  // that a later call could trip on.  Nothing else in the scratch has to
-  // start at a known value.
+  // Every call clears the whole zero region (exchange words and arrival
+  // counters, at the start of the scratch) before the layer's kernel runs --
+  // in the decode path's activation kernel, else with a memset -- so a call
+  // cut short (a timeout) leaves nothing that a later call could trip on.
+  // Nothing else in the scratch has to start at a known value.
+  if (linear_plan(M, K, N).sk &&
+      cudaMemsetAsync(scratch, 0, kWsZeroBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return W4A8_ERR_CUDA;
   w4a8_status st = prepare_impl(x, M, K, N, scratch, kStaticScratchBytes, stream, 0);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, scratch, kStaticScratchBytes, stream);
@@ -619,7 +679,8 @@ w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, vo
   unsigned long long* xch = reinterpret_cast<unsigned long long*>(ws + kChainZeroOff);
   unsigned* counters = reinterpret_cast<unsigned*>(ws + kChainZeroOff + kWsCntOff);
   float* slots = reinterpret_cast<float*>(ws + kChainSlotsOff);
-  const int warps_avail = (d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas) * kDecWarps;
+  const int ctas = d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas;  // the cooperative grid
+  const int warps_avail = ctas * kDecWarps;
   DecodeParams* host = new (std::nothrow) DecodeParams[size_t(n_layers)];
   if (!host) return W4A8_ERR_SHAPE;
   for (int64_t i = 0; i < n_layers; ++i) {
@@ -648,6 +709,7 @@ w4a8_status w4a8_chain_plan(const w4a8_chain_layer* layers, int64_t n_layers, vo
     p.W = p.U < warps_avail ? p.U : warps_avail;
     p.R = p.U / p.W;
     p.Rm = p.U % p.W;
+    one_token_split(p, ctas);
     host[i] = p;
   }
   // From pageable memory: the call returns once the table has been staged.
@@ -670,7 +732,7 @@ w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace, 
   if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return W4A8_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas));
-  cfg.blockDim = dim3(kDecThreads);
+  cfg.blockDim = dim3(kOneThreads);
   cfg.dynamicSmemBytes = dec_smem_bytes(1, kMaxK, true);
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -683,6 +745,167 @@ w4a8_status w4a8_chain_run(const void* plan, int64_t n_layers, void* workspace, 
   const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_chain_kernel, static_cast<const DecodeParams*>(plan),
                                            int(n_layers), static_cast<unsigned*>(workspace));
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ decode chains with fused activations
+
+namespace {
+
+constexpr int kActSets = 3;  // activation sets in rotation among producers
+
+struct ActSetLayout {
+  size_t rot_off, cnt_off, set_bytes, total;  // one set: [rot K_max fp32][cnt K_max/256 + amax]
+  int cnt_words;
+};
+
+ActSetLayout act_sets(int64_t kmax) {
+  ActSetLayout a{};
+  a.cnt_words = int(kmax / kRotBlock) + 1;  // block counters, then the absmax word
+  a.rot_off = 0;
+  a.cnt_off = round_up(size_t(kmax) * 4, 256);
+  a.set_bytes = round_up(a.cnt_off + size_t(a.cnt_words) * 4, 256);
+  a.total = a.set_bytes * kActSets;
+  return a;
+}
+
+// [0, kWsZeroBytes): exchange words and split-K counters (left at zero by
+// every layer); then the per-CTA partial slots; then the activation sets.
+constexpr size_t kDecChainSlotsOff = kWsZeroBytes;
+constexpr size_t kDecChainSetsOff = kDecChainSlotsOff + (size_t(2) * kDecMaxCtas * kDecTG * 16 * 4 + 255) / 256 * 256;
+
+struct ChainLink {
+  int producer = -1;   // the layer whose output this layer reads (fused), or -1
+  int64_t off = 0;     // producer: the outputs the consumers read start here
+  int64_t len = 0;     // and are this many (0: not a producer)
+  int set = -1;        // producer: its activation set
+  int zero_set = -1;   // this layer clears that set (the next layer produces into it)
+};
+
+// Which layers read which earlier layer's output, and the sets.
+void link_chain(const w4a8_chain_layer* L, int64_t n, ChainLink* link) {
+  for (int64_t i = 0; i < n; ++i) {
+    const uint16_t* x = L[i].x;
+    // the latest earlier layer whose output range overlaps this input
+    for (int64_t j = i - 1; j >= 0; --j) {
+      const uint16_t* y = L[j].y;
+      const bool overlaps = x < y + L[j].N && y < x + L[i].K;
+      if (!overlaps) continue;
+      const int64_t off = x - y;
+      const bool inside = off >= 0 && off % kRotBlock == 0 && off + L[i].K <= L[j].N;
+      if (inside && (link[j].len == 0 || (link[j].off == off && link[j].len == L[i].K))) {
+        link[j].off = off;
+        link[j].len = L[i].K;
+        link[i].producer = int(j);
+      }
+      break;
+    }
+  }
+  // sets in rotation; a set is cleared by the layer before its next producer,
+  // so every reader of the set's previous contents must come before that
+  std::vector<int64_t> producers;
+  for (int64_t i = 0; i < n; ++i)
+    if (link[i].len > 0) producers.push_back(i);
+  for (size_t a = 0; a < producers.size(); ++a) link[producers[a]].set = int(a % kActSets);
+  for (size_t a = 0; a + kActSets < producers.size(); ++a) {
+    const int64_t next = producers[a + kActSets];  // the next producer into this set
+    for (int64_t c = next - 1; c < n; ++c)
+      if (link[c].producer == producers[a]) link[c].producer = -1;  // would read a cleared set: use x
+  }
+  for (size_t a = kActSets; a < producers.size(); ++a) link[producers[a] - 1].zero_set = link[producers[a]].set;
+}
+
+}  // namespace
+
+size_t w4a8_decode_chain_workspace_bytes(const w4a8_chain_layer* layers, int64_t n_layers) {
+  if (!layers || n_layers < 1) return 0;
+  int64_t kmax = 0;
+  for (int64_t i = 0; i < n_layers; ++i) {
+    if (!weight_shape_ok(layers[i].N, layers[i].K)) return 0;
+    kmax = layers[i].K > kmax ? layers[i].K : kmax;
+  }
+  return kDecChainSetsOff + act_sets(kmax).total;
+}
+
+w4a8_status w4a8_decode_chain(const w4a8_chain_layer* layers, int64_t n_layers, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!layers || !workspace) return W4A8_ERR_NULL;
+  if (n_layers < 1 || n_layers > (int64_t(1) << 20)) return W4A8_ERR_SHAPE;
+  int64_t kmax = 0;
+  for (int64_t i = 0; i < n_layers; ++i) {
+    const w4a8_chain_layer& L = layers[i];
+    if (!L.packed || !L.x || !L.y) return W4A8_ERR_NULL;
+    if (!weight_shape_ok(L.N, L.K)) return W4A8_ERR_SHAPE;
+    if (!aligned16(L.packed) || !aligned16(L.x) || !aligned16(L.y)) return W4A8_ERR_ALIGN;
+    kmax = L.K > kmax ? L.K : kmax;
+  }
+  if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+  if (workspace_bytes < w4a8_decode_chain_workspace_bytes(layers, n_layers)) return W4A8_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<ChainLink> link(static_cast<size_t>(n_layers));
+  link_chain(layers, n_layers, link.data());
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const ActSetLayout A = act_sets(kmax);
+  uint8_t* sets = ws + kDecChainSetsOff;
+  auto set_rot = [&](int k) { return reinterpret_cast<float*>(sets + k * A.set_bytes + A.rot_off); };
+  auto set_cnt = [&](int k) { return reinterpret_cast<unsigned*>(sets + k * A.set_bytes + A.cnt_off); };
+  // every set's counters and absmax start at zero
+  for (int k = 0; k < kActSets; ++k)
+    if (cudaMemsetAsync(set_cnt(k), 0, size_t(A.cnt_words) * 4, s) != cudaSuccess) return W4A8_ERR_CUDA;
+  const int ctas = d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas;
+  for (int64_t i = 0; i < n_layers; ++i) {
+    const w4a8_chain_layer& L = layers[i];
+    const PackedLayout PL = packed_layout(L.N, L.K);
+    const uint8_t* pk = static_cast<const uint8_t*>(L.packed);
+    DecodeParams p{};
+    p.x = L.x;
+    p.units = pk + PL.off_units;
+    p.sch = reinterpret_cast<const float*>(pk + PL.off_sch);
+    p.cb = reinterpret_cast<const float*>(pk + PL.off_cb);
+    p.y = L.y;
+    p.slots = reinterpret_cast<float*>(ws + kDecChainSlotsOff);
+    p.xch = reinterpret_cast<unsigned long long*>(ws);
+    p.counters = reinterpret_cast<unsigned*>(ws + kWsCntOff);
+    p.err = d->err;
+    p.M = 1;
+    p.N = int(L.N);
+    p.K = int(L.K);
+    p.C = int(L.K / kChunkK);
+    p.T = int(L.N / kTileRows);
+    p.P = (p.T + kDecTG - 1) / kDecTG;
+    p.U = p.P * p.C;
+    p.W = p.U < ctas * kDecWarps ? p.U : ctas * kDecWarps;
+    p.R = p.U / p.W;
+    p.Rm = p.U % p.W;
+    one_token_split(p, ctas);
+    const ChainLink& k = link[size_t(i)];
+    if (k.len > 0) {
+      p.act_rot = set_rot(k.set);
+      p.act_cnt = set_cnt(k.set);
+      p.act_amax = set_cnt(k.set) + (A.cnt_words - 1);
+      p.act_off = int(k.off);
+      p.act_len = int(k.len);
+    }
+    if (k.producer >= 0) {
+      const int ps = link[size_t(k.producer)].set;
+      p.in_rot = set_rot(ps);
+      p.in_amax = set_cnt(ps) + (A.cnt_words - 1);
+    }
+    if (k.zero_set >= 0) {
+      p.zero_cnt = set_cnt(k.zero_set);
+      p.zero_n = A.cnt_words;
+    }
+    const size_t smem = dec_smem_bytes(1, p.K, true);
+    cudaError_t e;
+    if (!p.in_rot && p.K > kDecPairK)
+      e = launch_pdl_cluster(decode_one_kernel<true>, dim3((unsigned(p.G) + 1) & ~1u), dim3(kOneThreads), 2, smem, s,
+                             p);
+    else
+      e = launch_pdl(decode_one_kernel<true>, dim3(unsigned(p.G)), dim3(kOneThreads), smem, s, p);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+  }
+  return W4A8_OK;
 }
 
 // ------------------------------------------------------------------ fidelity checks
