@@ -378,6 +378,19 @@ C3_SHAPES = (("qkv", 5120, 10240), ("out", 5120, 5120), ("gate", 5120, 17408), (
              ("down", 17408, 5120))
 
 
+def c2_path(m: int, k: int, n: int) -> str:
+    """Which kernel w4a8_linear runs for (M, K, N) (the library's rule)."""
+    if m == 1:
+        return "one-token decode (activation step fused)"
+    if 64 <= m <= 128 and (n + 127) // 128 < 100:
+        return "small-batch tensor-core (stream-K)"
+    if m <= 16:
+        return "decode"
+    if m <= 64:
+        return "decode, slices of 16"
+    return "tensor-core GEMM"
+
+
 def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
     """Down-projection shape K=17408, N=5120 at several token counts, 8 weight
     copies cycled: M <= 64 runs the decode kernel (one launch per 16 tokens),
@@ -414,7 +427,7 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
         us = e0.elapsed_time(e1) * 1e3 / st
         out[f"M={m}"] = {"us_per_call": us, "weight_GBs": wbytes / us / 1e3,
                          "us_per_token": us / m,
-                         "path": "decode" if m <= 16 else "decode, slices of 16" if m <= 64 else "tensor-core GEMM"}
+                         "path": c2_path(m, k, n)}
         del replay
     del copies
     torch.cuda.empty_cache()
@@ -965,15 +978,15 @@ def main() -> None:
             "launch": "timed steps replayed from CUDA graphs (1 kernel per step, programmatic dependent launch)",
         },
         "roofline": {
-            "kernel": "decode_kernel<1,4,1,1> (M=1, rotate + quantise fused)",
+            "kernel": "decode_one_kernel<true> (M=1, rotate + quantise fused)",
             "bound": "hbm", "achieved": step_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": step_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
-            "traffic": profiled_traffic("decode_kernel_fused", ["gemv.cuh", "act.cuh", "common.cuh"]),
+            "traffic": profiled_traffic("decode_one_kernel_fused", ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"]),
             "us_per_launch": ms_step * 1e3,
             "note": "the step is this one kernel, so its launch duration is the step time",
         },
         "decode_run_only": {
-            "kernel": "decode_kernel<1,4,1,0> (activations prepared once, runs back to back)",
+            "kernel": "decode_one_kernel<false> (activations prepared once, runs back to back)",
             "achieved": achieved, "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
             "us_per_launch": gemv_ms * 1e3,
         },

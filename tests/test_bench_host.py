@@ -21,9 +21,12 @@ def test_weight_bytes_is_the_packed_layer():
 def test_committed_traffic_matches_its_source_hash():
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         d = json.load(f)
-    files = {"decode_kernel_fused": ["gemv.cuh", "act.cuh", "common.cuh"],
+    files = {"decode_one_kernel_fused": ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"],
              "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"]}
     for kernel, srcs in files.items():
+        if kernel not in d:
+            assert bench.profiled_traffic(kernel, srcs) is None
+            continue
         got = bench.profiled_traffic(kernel, srcs)
         if d[kernel]["source_sha256_16"] == bench.kernel_source_hash(srcs):
             assert got == pytest.approx(d[kernel]["dram_bytes_per_launch"])
@@ -65,3 +68,13 @@ def test_oracle_pool_splits_rows_over_processes():
     finally:
         pool.close()
     assert np.isfinite(bench.weight_bytes(48, 256))
+
+
+def test_c2_path_names_follow_the_library_rule():
+    assert bench.c2_path(1, 17408, 5120).startswith("one-token")
+    assert bench.c2_path(4, 17408, 5120) == "decode"
+    assert bench.c2_path(32, 17408, 5120) == "decode, slices of 16"
+    assert bench.c2_path(64, 17408, 5120).startswith("small-batch")
+    assert bench.c2_path(128, 17408, 5120).startswith("small-batch")
+    assert bench.c2_path(128, 5120, 17408) == "tensor-core GEMM"
+    assert bench.c2_path(256, 17408, 5120) == "tensor-core GEMM"

@@ -61,7 +61,6 @@ constexpr size_t kWsZeroBytes = (kWsXchBytes + size_t(kDecMaxCtas) * 4 + 255) / 
 constexpr size_t kDecSmemBase = 2 * 65536;         // room for a 64 KiB-aligned 64 KiB table
 constexpr int kDecSchRows = 1024;                  // row scales staged in shared memory per CTA
 // Units in flight per warp (register ring depth) per variant.
-constexpr int kDecDepthSingle = 4;                 // one token (one quad of units, see decode_body)
 constexpr int kDecDepth1 = 3;                      // 2..8 tokens
 constexpr int kDecDepth2 = 2;                      // 9..16 tokens
 
@@ -162,11 +161,11 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 
 // Per-unit registers: index bytes and group scales of the two tiles, and (for
 // more than one token) the B fragments of the unit's chunk.
-template <int NB, bool SINGLE>
+template <int NB>
 struct DecStage {
   uint4 w[kDecTG];
   uint2 s[kDecTG];
-  uint4 x[SINGLE ? 1 : NB][2];
+  uint4 x[NB][2];
 };
 
 __device__ __forceinline__ uint4 ld_stream_v4(const uint8_t* p) {
@@ -189,43 +188,34 @@ __device__ __forceinline__ uint2 ld_stream_v2(const uint8_t* p) {
 
 // A lane's index words and scale codes of one unit: wp points at the lane's
 // 16 index bytes of tile 0 in the unit, sp at its 8 scale bytes of tile 0.
-// (For one token, sp points at the lane's 4 scale bytes, see dec_compute_one.)
-template <int NB, bool SINGLE>
-__device__ __forceinline__ void dec_load_w(DecStage<NB, SINGLE>& st, const uint8_t* wp, const uint8_t* sp) {
+template <int NB>
+__device__ __forceinline__ void dec_load_w(DecStage<NB>& st, const uint8_t* wp, const uint8_t* sp) {
   st.w[0] = ld_stream_v4(wp);
   st.w[1] = ld_stream_v4(wp + kChunkIdxBytes);
-  if constexpr (SINGLE) {
-    st.s[0].x = ld_stream_u32(sp);
-    st.s[1].x = ld_stream_u32(sp + kChunkSrelBytes);
-  } else {
-    st.s[0] = ld_stream_v2(sp);
-    st.s[1] = ld_stream_v2(sp + kChunkSrelBytes);
-  }
+  st.s[0] = ld_stream_v2(sp);
+  st.s[1] = ld_stream_v2(sp + kChunkSrelBytes);
 }
 
-template <int NB, bool SINGLE>
-__device__ __forceinline__ void dec_load_x(DecStage<NB, SINGLE>& st, const DecodeParams& p, int c, int lane) {
-  if constexpr (!SINGLE) {
+template <int NB>
+__device__ __forceinline__ void dec_load_x(DecStage<NB>& st, const DecodeParams& p, int c, int lane) {
 #pragma unroll
-    for (int j = 0; j < NB; ++j) {
-      if ((lane >> 2) + 8 * j < p.M) {
-        const uint4* src = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
-        st.x[j][0] = __ldg(src);
-        st.x[j][1] = __ldg(src + 1);
-      } else {
-        st.x[j][0] = make_uint4(0, 0, 0, 0);
-        st.x[j][1] = make_uint4(0, 0, 0, 0);
-      }
+  for (int j = 0; j < NB; ++j) {
+    if ((lane >> 2) + 8 * j < p.M) {
+      const uint4* src = p.xfrag + (size_t(c * NB + j) * 32 + lane) * 2;
+      st.x[j][0] = __ldg(src);
+      st.x[j][1] = __ldg(src + 1);
+    } else {
+      st.x[j][0] = make_uint4(0, 0, 0, 0);
+      st.x[j][1] = make_uint4(0, 0, 0, 0);
     }
   }
 }
 
-// One unit: all 32 table lookups (and, for one token, the 4 B fragments from
-// shared memory) are issued first, back to back, so their latencies overlap;
-// then the 8 (x NB) MMAs and the fp32 group-scale accumulation.
-template <int NB, bool SINGLE>
-__device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, float (&acc)[kDecTG][NB][4],
-                                            uint32_t lut_lane, uint32_t xs_chunk) {
+// One unit: all 32 table lookups are issued first, back to back, so their
+// latencies overlap; then the 8 x NB MMAs and the fp32 group-scale
+// accumulation.
+template <int NB>
+__device__ __forceinline__ void dec_compute(const DecStage<NB>& st, float (&acc)[kDecTG][NB][4], uint32_t lut_lane) {
   const float zero = 0.f;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {  // two halves of two k16 steps each
@@ -244,22 +234,14 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, floa
       }
     }
     uint32_t b[2][NB][2];
-    if constexpr (SINGLE) {
-      const uint4 v = lds128_(xs_chunk + 16u * h);
-      b[0][0][0] = v.x;
-      b[0][0][1] = v.y;
-      b[1][0][0] = v.z;
-      b[1][0][1] = v.w;
-    } else {
 #pragma unroll
-      for (int s2 = 0; s2 < 2; ++s2)
+    for (int s2 = 0; s2 < 2; ++s2)
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          const uint4& xv = st.x[j][h];
-          b[s2][j][0] = s2 ? xv.z : xv.x;
-          b[s2][j][1] = s2 ? xv.w : xv.y;
-        }
-    }
+      for (int j = 0; j < NB; ++j) {
+        const uint4& xv = st.x[j][h];
+        b[s2][j][0] = s2 ? xv.z : xv.x;
+        b[s2][j][1] = s2 ? xv.w : xv.y;
+      }
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
       const int s = 2 * h + s2;
@@ -273,52 +255,9 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB, SINGLE>& st, floa
           mma_16816z(d, a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b[s2][j][0], b[s2][j][1], zero);
           acc[i][j][0] = fmaf(d[0], sc.x, acc[i][j][0]);
           acc[i][j][2] = fmaf(d[2], sc.y, acc[i][j][2]);
-          if (!SINGLE) {
-            acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
-            acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
-          }
+          acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
+          acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
         }
-      }
-    }
-  }
-}
-
-// One token, one unit (chunk c): the 32 table lookups, then the 8 MMAs
-// into dm, the fragment shared by the chunk pair (c & ~1, c | 1).  Column n
-// of dm is group n & 3 of chunk (c & ~1) + (n >> 2).  In step s of chunk c
-// only lane (g, t) with g = 4 (c & 1) + s has a non-zero B fragment: x of
-// that group, k = 64 c + 16 s + 2 t (+1) and + 8 (+9).  xv holds that pair
-// for the lane's own chunk of the pair (parity g >> 2), and bm[s] is all
-// ones where step s of this unit's chunk is the lane's.  FIRST: the unit
-// opens the pair, so its first step starts the fragment from zero.
-template <int NB, bool SINGLE, bool FIRST>
-__device__ __forceinline__ void dec_compute_one(const DecStage<NB, SINGLE>& st, float (&dm)[kDecTG][4],
-                                                uint32_t lut_lane, uint2 xv, const uint32_t (&bm)[4]) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t a[kDecTG][2][4];
-#pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int s = 2 * h + s2;
-#pragma unroll
-      for (int i = 0; i < kDecTG; ++i) {
-        const uint32_t word = s == 0 ? st.w[i].x : s == 1 ? st.w[i].y : s == 2 ? st.w[i].z : st.w[i].w;
-        a[i][s2][0] = lds32(prmt(word, lut_lane, 0x7604u));
-        a[i][s2][1] = lds32(prmt(word, lut_lane, 0x7614u));
-        a[i][s2][2] = lds32(prmt(word, lut_lane, 0x7624u));
-        a[i][s2][3] = lds32(prmt(word, lut_lane, 0x7634u));
-      }
-    }
-#pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int s = 2 * h + s2;
-      const uint32_t b0 = xv.x & bm[s], b1 = xv.y & bm[s];
-#pragma unroll
-      for (int i = 0; i < kDecTG; ++i) {
-        if (FIRST && s == 0)
-          mma_16816z(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1, 0.f);
-        else
-          mma_16816(dm[i], a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b0, b1);
       }
     }
   }
@@ -418,81 +357,6 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 }
 
-// One token: a pair split between warps (levels 2 and 3 of the reduction);
-// CTAs cf..cl hold parts of it.  Lane l owns row l of the pair (row 16 i + g + 8 h of the partial layout):
-// it adds the contributing warps' partials in warp order.  A pair that also
-// spans another CTA is finished by whichever of its CTAs comes second:
-//  * two CTAs (the usual case): each lane swaps its CTA's sum, tagged, into
-//    the row's exchange word with one 64-bit atomic; a lane that gets the
-//    other CTA's tagged sum back adds it, writes y and clears the word.  A
-//    sum of two fp32 terms is the same in either order, so the result does
-//    not depend on which CTA arrives first;
-//  * more CTAs: each parks its sum in the workspace and counts itself in with
-//    one acquire-release atomic by lane 0; the last to arrive adds the CTAs'
-//    sums in CTA order and writes y.
-__device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, int q0, int q1, int v0, int v1,
-                                               int cf, int cl, const int (&wb)[kDecWarps + 1], uint32_t parts,
-                                               uint32_t part_bytes, int lane, const DecEpi& ep) {
-  float tot = 0.f;
-#pragma unroll
-  for (int ww = 0; ww < kDecWarps; ++ww) {
-    const bool holds = (wb[ww] < q1) & (wb[ww + 1] > q0) & (wb[ww] < wb[ww + 1]);
-    const uint32_t slot = parts + uint32_t(ww * 2 + (wb[ww] >= q0 ? 0 : 1)) * part_bytes;
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(slot + uint32_t(lane) * 4u));
-    tot = holds ? tot + v : tot;
-  }
-  const int row = pr * (kDecTG * 16) + lane;
-  if (!(q0 >= v0 && q1 <= v1)) {
-    // level 3: the pair spans CTAs cf..cl
-    if (cl == cf + 1) {
-      unsigned long long* word = p.xch + size_t(cf) * 32 + lane;
-      unsigned long long other;
-      asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;"
-                   : "=l"(other)
-                   : "l"(word), "l"((1ull << 32) | __float_as_uint(tot))
-                   : "memory");
-      if ((other >> 32) == 0) return;  // the other CTA finishes this row
-      *word = 0ull;                    // ready for the next launch on this workspace
-      tot += __uint_as_float(unsigned(other));
-    } else {
-      const int sf = dec_slot_floats(1);
-      p.slots[size_t(blockIdx.x * 2 + (v0 >= q0 ? 0 : 1)) * sf + lane] = tot;
-      __syncwarp();
-      unsigned old = 0;
-      if (lane == 0)
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + cf) : "memory");
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old != unsigned(cl - cf)) return;  // another CTA finishes this pair
-      __syncwarp();  // the other lanes' loads come after lane 0's acquire
-      tot = 0.f;
-      for (int c0 = cf; c0 <= cl; c0 += 4) {
-        float v[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int cc = c0 + r;
-          const bool have = cc <= cl;
-          v[r] = have ? __ldcg(p.slots + size_t(cc * 2 + (dec_cta_begin<kDecWarps>(cc, p) >= q0 ? 0 : 1)) * sf + lane)
-                      : 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) tot += v[r];
-      }
-      if (lane == 0) p.counters[cf] = 0u;  // ready for the next launch on this workspace
-    }
-  }
-  if (row < p.N) {
-    const int rr = row - ep.row0;
-    float sc, sx;
-    if (rr < kDecSchRows)
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(ep.sch + uint32_t(rr) * 4u));
-    else
-      sc = __ldg(p.sch + row);
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sx) : "r"(ep.sx));
-    p.y[row] = __bfloat16_as_ushort(__float2bfloat16_rn(tot * sc * sx));
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Work split ("stream-K"): the P * C units, in the order they lie in memory,
 // are cut into W equal ranges, one per warp; a CTA's 16 warps hold 16
@@ -503,41 +367,26 @@ __device__ __forceinline__ void dec_reduce_one(const DecodeParams& p, int pr, in
 // fixed order (the result is deterministic): the warps of a CTA leave their
 // partials in shared memory and one warp adds them after a CTA barrier; a
 // pair that also crosses into other CTAs is finished by the CTA that comes
-// last to it (dec_reduce_one for one token, the counter path below for
-// more).
-//
-// FUSED (one token): the kernel also does the activation step: every CTA
-// rotates the bf16 row and quantises it to int8 (the activation kernel's
-// arithmetic, so the codes and s_x are the same bits).  A warp keeps its
-// first few rotated 256-blocks in registers until the row's absmax is known
-// and quantises them from there; blocks past those are rotated again.
-// Launched as clusters of two CTAs, each CTA of a pair rotates and
-// quantises every other 256-block and writes its codes into both CTAs'
-// shared memory.  One launch then makes the whole layer.
-//
-// The body is a device function so that a persistent kernel can run a chain
-// of layers with it; `wait_inputs` is where the body waits for what an
-// earlier step wrote (the activations, and the workspace it reuses).
+// last to it (an arrival counter; the last CTA adds the partials in CTA
+// order).  This kernel serves 2..16 tokens per launch; one token runs the
+// kernel in gemv1.cuh.
 struct DecWaitPdl {
   static constexpr int kLoadsAhead = 4;  // kept blocks whose loads are all issued before the first transform
   __device__ __forceinline__ void operator()() const { pdl_wait(); }
 };
 
-template <int NB, int D, bool SINGLE, bool FUSED, class Wait>
+template <int NB, int D, class Wait>
 __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& wait_inputs) {
-  static_assert(!FUSED || SINGLE, "the fused activation step handles one token");
-  constexpr int kW = dec_warps(SINGLE);
+  constexpr int kW = dec_warps(false);
   constexpr int kThr = kW * 32;
   extern __shared__ __align__(16) uint8_t dec_smem[];
   const uint32_t base = smem_u32(dec_smem);
   const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;  // 64 KiB aligned: bits 8..15 are zero
-  const uint32_t xs = lut + 65536u;                   // one token: x staged here (2 K bytes)
-  const uint32_t parts = xs + (SINGLE ? uint32_t(p.C) * 128u : 0u);  // [warp][2] partials
+  const uint32_t parts = lut + 65536u;                // [warp][2] partials
   const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
   const uint32_t sch_s = parts + uint32_t(kW * 2) * part_bytes;  // row scales
   const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
   const uint32_t wbeg_s = sx_s + 64;  // warp range starts [17]; at +96 the CTA pair context [4]
-  const uint32_t red_s = wbeg_s + 128;                                    // per-warp maxima [16]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int cta_w0 = blockIdx.x * kW;
   const int w = cta_w0 + wl;
@@ -550,31 +399,20 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   // This lane's index bytes and scale bytes in unit u0; every later unit is
   // kUnitBytes further on.
   const uint8_t* wp = p.units + size_t(u0) * kUnitBytes + lane * 16;
-  const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8 +
-                      (SINGLE ? 4 * (lane & 1) : 0);
+  const uint8_t* sp = p.units + size_t(u0) * kUnitBytes + 2 * kChunkIdxBytes + (lane >> 2) * 8;
 
   // The codebook level this lane puts in the table: loaded ahead of the
   // weight stream so that it does not queue behind it.
   const float level = p.cb[lane & 15];
 
-  DecStage<NB, SINGLE> st[D];
+  DecStage<NB> st[D];
   // Weights do not depend on the previous kernel: start streaming them now,
-  // before the wait.  (x for more than one token comes from it, so it is
-  // loaded after the wait.)
-  if constexpr (SINGLE) {
-    // one token: slot d holds the next unit u with u % D == d (see the loop below)
+  // before the wait.  (x comes from it, so it is loaded after the wait.)
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int off = ((d - u0) % D + D) % D;  // units from u0 to the first one with residue d
-      if (off < n_units) dec_load_w<NB, SINGLE>(st[d], wp + off * kUnitBytes, sp + off * kUnitBytes);
-    }
-  } else {
-#pragma unroll
-    for (int d = 0; d < D; ++d)
-      if (d < n_units) dec_load_w<NB, SINGLE>(st[d], wp + d * kUnitBytes, sp + d * kUnitBytes);
-    wp += D * kUnitBytes;
-    sp += D * kUnitBytes;
-  }
+  for (int d = 0; d < D; ++d)
+    if (d < n_units) dec_load_w<NB>(st[d], wp + d * kUnitBytes, sp + d * kUnitBytes);
+  wp += D * kUnitBytes;
+  sp += D * kUnitBytes;
 
   // The CTA's range, its warps' range starts and its rows' scales (all
   // independent of the previous kernel).
@@ -617,128 +455,14 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
                  "r"(*reinterpret_cast<const uint32_t*>(&h)));
   }
   wait_inputs();  // activations, scales and counters come from an earlier step
-  int cx = first_c;  // chunk of the next x fragment to load (more than one token)
-  if constexpr (FUSED) {
-    // Rotate the row (warp per 256-block) and find its absmax.  Launched as
-    // clusters of two CTAs, each CTA of a pair takes every other 256-block:
-    // the pair swaps its maxima and each CTA writes its half of the codes
-    // into both CTAs' shared memory (launched without clusters, a CTA takes
-    // all blocks).
-    const uint32_t crank = cluster_ctarank(), ncta = cluster_nctarank();
-    const int nblk = p.K / kRotBlock;
-    const int nown = (nblk - int(crank) + int(ncta) - 1) / int(ncta);  // blocks crank + ncta j
-    // A warp keeps the rotated values of its first kKeep blocks in registers
-    // until the absmax is known; blocks past those are rotated again.
-    constexpr int kKeep = 4;
-    float amax = 0.f;
-    float vk[kKeep][8];
-    // the first kLoadsAhead kept blocks' loads are in flight before the first transform
-    constexpr int kAhead = Wait::kLoadsAhead < kKeep ? Wait::kLoadsAhead : kKeep;
-    uint4 raw[kAhead];
+  int cx = first_c;  // chunk of the next x fragment to load
+  if (threadIdx.x < p.M)
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + threadIdx.x * 4u), "f"(p.s_x[threadIdx.x]));
 #pragma unroll
-    for (int jj = 0; jj < kAhead; ++jj) {
-      const int j = wl + kW * jj;
-      if (j < nown) raw[jj] = load_block_lane(p.x, int(crank) + int(ncta) * j, lane);
-    }
-    // The warp's next 8 units (after the 4 in its register ring) into L2 with
-    // one bulk prefetch, issued behind the token's loads: the memory system
-    // streams them while the CTA rotates and quantises the token.
-    {
-      const int pa = min(u0 + D, u1), pb = min(u0 + 3 * D, u1);
-      if (lane == 0 && pb > pa)
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.units + size_t(pa) * kUnitBytes),
-                     "r"(uint32_t(pb - pa) * uint32_t(kUnitBytes))
-                     : "memory");
-    }
-#pragma unroll
-    for (int jj = 0; jj < kKeep; ++jj) {
-      const int j = wl + kW * jj;
-      if (j < nown) {
-        rotate_words_lane(jj < kAhead ? raw[jj] : load_block_lane(p.x, int(crank) + int(ncta) * j, lane), lane,
-                          vk[jj]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(vk[jj][i]));
-      }
-    }
-    for (int j = wl + kW * kKeep; j < nown; j += kW) {
-      float v[8];
-      rotate_block_lane(p.x, int(crank) + int(ncta) * j, lane, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(red_s + uint32_t(wl) * 4u), "f"(amax));
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kW; ++i) {
-      float m;
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(m) : "r"(red_s + uint32_t(i) * 4u));
-      amax = fmaxf(amax, m);
-    }
-    uint32_t peer_xs = 0;
-    if (ncta > 1) {
-      // this CTA's maximum goes to s_x[1]'s slot (one token: unused), read by the partner
-      if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + 4u), "f"(amax));
-      cluster_sync_all();
-      amax = fmaxf(amax, ld_cluster_f32(sx_s + 4u, crank ^ 1u));
-      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(peer_xs) : "r"(xs), "r"(crank ^ 1u));
-    }
-    const float s = quant_scale(amax);
-    const QuantScale qs = quant_prepare(s);
-    if (threadIdx.x == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s), "f"(s));
-    // Codes as fp16 in the B-fragment order: the pair (k, k + 1) of chunk c,
-    // k16 step s4, half w, lane t sits at c 128 + t 32 + (2 s4 + w) 4; a run
-    // of 8 values from k0 (a multiple of 8) covers t = 0..3.
-    auto put_codes = [&](auto fast, int k0, const float (&v)[8]) {
-      constexpr bool kFast = decltype(fast)::value;
-      const uint32_t off = uint32_t(k0 >> 6) * 128u + uint32_t(2 * ((k0 >> 4) & 3) + ((k0 >> 3) & 1)) * 4u;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const __half2 h = __floats2half2_rn(quant_code<kFast>(v[2 * t], qs), quant_code<kFast>(v[2 * t + 1], qs));
-        const uint32_t hv = *reinterpret_cast<const uint32_t*>(&h);
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(xs + off + uint32_t(t) * 32u), "r"(hv));
-        if (ncta > 1) asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(peer_xs + off + uint32_t(t) * 32u), "r"(hv));
-      }
-    };
-    auto quantise = [&](auto fast) {
-#pragma unroll
-      for (int jj = 0; jj < kKeep; ++jj) {
-        const int j = wl + kW * jj;
-        if (j < nown) put_codes(fast, (int(crank) + int(ncta) * j) * kRotBlock + lane * 8, vk[jj]);
-      }
-      for (int j = wl + kW * kKeep; j < nown; j += kW) {
-        float v[8];
-        const int b = int(crank) + int(ncta) * j;
-        rotate_block_lane(p.x, b, lane, v);
-        put_codes(fast, b * kRotBlock + lane * 8, v);
-      }
-    };
-    if (qs.fast)
-      quantise(std::true_type{});
-    else
-      quantise(std::false_type{});
-    if (ncta > 1) cluster_sync_all();  // both halves of the codes are in place; no remote access after this
-  } else {
-    if (threadIdx.x < p.M)
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_s + threadIdx.x * 4u), "f"(p.s_x[threadIdx.x]));
-    if constexpr (SINGLE) {
-      // token 0's B fragments: per chunk, lanes t = 0..3 of the fragment layout (128 bytes)
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(p.xfrag);
-      for (int e = threadIdx.x; e < p.C * 8; e += kThr) {
-        const int c = e >> 3, qq = e & 7;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + size_t(c) * 1024 + qq * 16));
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xs + uint32_t(c) * 128u + uint32_t(qq) * 16u),
-                     "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
-      }
-    } else {
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        if (d < n_units) {
-          dec_load_x<NB, SINGLE>(st[d], p, cx, lane);
-          if (++cx == p.C) cx = 0;
-        }
-      }
+  for (int d = 0; d < D; ++d) {
+    if (d < n_units) {
+      dec_load_x<NB>(st[d], p, cx, lane);
+      if (++cx == p.C) cx = 0;
     }
   }
 #pragma unroll
@@ -749,69 +473,13 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   __syncthreads();
 
   const uint32_t lut_lane = lut + uint32_t(lane) * 4u;
-  const uint32_t xs_lane = xs + uint32_t(lane & 3) * 32u;
   float acc[kDecTG][NB][4];
   dec_zero<NB>(acc);
-  // One token: dm is the MMA fragment of the current chunk pair (columns =
-  // its 8 groups), ga the fp32 sums of dm * s_rel (rows g, g + 8 x groups
-  // 2 t, 2 t + 1 of each pair).  sr_e / sr_o hold the lane's 4 scale codes
-  // of the pair's even / odd chunk, bytes (row g, group 2 (t & 1)),
-  // (row g + 8, same), (row g, group + 1), (row g + 8, group + 1); lanes
-  // t < 2 apply the even chunk's, t >= 2 the odd one's.  bm_e / bm_o: the
-  // lane's B-fragment masks per k16 step for even / odd chunks.
-  float dm[kDecTG][4], ga[kDecTG][4];
-  uint32_t sr_e[kDecTG], sr_o[kDecTG], bm_e[4], bm_o[4];
-  const int g_lane = lane >> 2, t_lane = lane & 3;
-#pragma unroll
-  for (int i = 0; i < kDecTG; ++i) {
-    sr_e[i] = sr_o[i] = 0u;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dm[i][e] = ga[i][e] = 0.f;
-  }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    bm_e[q] = (g_lane == q) ? 0xFFFFFFFFu : 0u;      // even chunks: lanes g = 0..3
-    bm_o[q] = (g_lane == 4 + q) ? 0xFFFFFFFFu : 0u;  // odd chunks: lanes g = 4..7
-  }
-  // the lane's x pair in the chunk of its parity, relative to the pair's even chunk
-  const uint32_t xb_lane = xs_lane + uint32_t(g_lane & 3) * 8u + uint32_t(g_lane >> 2) * 128u;
-  // Lanes t < 2 hold columns of the even chunk, t >= 2 those of the odd one.
-  auto scale_pair = [&]() {
-#pragma unroll
-    for (int i = 0; i < kDecTG; ++i) {
-      const uint32_t sr = t_lane < 2 ? sr_e[i] : sr_o[i];
-      const float2 s02 = e4m3x2_to_float2(sr);
-      const float2 s13 = e4m3x2_to_float2(sr >> 16);
-      ga[i][0] = fmaf(dm[i][0], s02.x, ga[i][0]);
-      ga[i][2] = fmaf(dm[i][2], s02.y, ga[i][2]);
-      ga[i][1] = fmaf(dm[i][1], s13.x, ga[i][1]);
-      ga[i][3] = fmaf(dm[i][3], s13.y, ga[i][3]);
-    }
-  };
-  // Row sums over the lane's group columns and the 4 lanes of a row; the
-  // totals go to acc[i][0][0] (row g) and acc[i][0][2] (row g + 8), token 0.
-  auto finish_rows = [&]() {
-#pragma unroll
-    for (int i = 0; i < kDecTG; ++i) {
-      float r0 = ga[i][0] + ga[i][1], r1 = ga[i][2] + ga[i][3];
-      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
-      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-      r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
-      r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
-      acc[i][0][0] = r0;
-      acc[i][0][2] = r1;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ga[i][e] = 0.f;
-    }
-  };
   int cur_pair = first_pair, cur_c = first_c, c_first = first_c;
-  auto compute = [&](const DecStage<NB, SINGLE>& s) {  // 2..16 tokens (one token: the quad loop below)
-    if constexpr (!SINGLE) dec_compute<NB, SINGLE>(s, acc, lut_lane, xs_lane + uint32_t(cur_c) * 128u);
-  };
+  auto compute = [&](const DecStage<NB>& s) { dec_compute<NB>(s, acc, lut_lane); };
   // A finished or range-ending pair: write y if this warp covered all of it,
   // else park the partial in shared memory (slot 0: the warp's first pair).
   auto close_pair = [&](int c_last) {
-    if constexpr (SINGLE) finish_rows();
     if (c_first == 0 && c_last == p.C - 1) {
       dec_epilogue<NB>(acc, p, cur_pair, lane, ep);
     } else {
@@ -828,79 +496,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
       c_first = 0;
     }
   };
-  auto refill = [&](DecStage<NB, SINGLE>& s, int off_units) {
-    dec_load_w<NB, SINGLE>(s, wp + off_units * kUnitBytes, sp + off_units * kUnitBytes);
-    if constexpr (!SINGLE) {
-      dec_load_x<NB, SINGLE>(s, p, cx, lane);
-      if (++cx == p.C) cx = 0;
-    }
+  auto refill = [&](DecStage<NB>& s, int off_units) {
+    dec_load_w<NB>(s, wp + off_units * kUnitBytes, sp + off_units * kUnitBytes);
+    dec_load_x<NB>(s, p, cx, lane);
+    if (++cx == p.C) cx = 0;
   };
-  if constexpr (SINGLE) {
-    // Quads: the 4 consecutive units 4 q .. 4 q + 3 are 4 chunks of one tile
-    // pair (C is a multiple of 4), i.e. two chunk pairs.  The ring holds
-    // kQ = D / 4 quads: unit 4 q + d sits in slot 4 (q mod kQ) + d and the
-    // slot is refilled with unit 4 (q + kQ) + d.  Units outside the warp's
-    // range are skipped (the first and last quads only).  A pair is closed
-    // once per quad at most.
-    static_assert(!SINGLE || D % 4 == 0, "one token: the ring holds whole quads");
-    constexpr int kQ = D / 4;  // quads in flight
-    const int q0 = u0 >> 2, q_end = n_units > 0 ? ((u1 - 1) >> 2) + 1 : q0;
-    int cq = cur_c & ~3;
-    // One quad q: its units sit in slots 4 r + d (r = q % kQ); each is
-    // refilled with the unit kQ quads further on.
-    auto quad = [&](auto R, int q) {
-      constexpr int r = decltype(R)::value;
-      if (q < q0 || q >= q_end) return;
-      const int lo = u0 - 4 * q, hi = u1 - 4 * q;  // units 4 q + d with lo <= d < hi are the warp's
-      const uint8_t* wq = wp + (4 * q - u0) * kUnitBytes;  // this lane's bytes in unit 4 q
-      const uint8_t* sq = sp + (4 * q - u0) * kUnitBytes;
-      const uint32_t xq = xb_lane + uint32_t(cq) * 128u;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {  // chunk pair (cq + 2 j, cq + 2 j + 1)
-        const uint2 xv = lds64(xq + 256u * j);
-        const int de = 2 * j, dd = 2 * j + 1;
-        if (de >= lo && de < hi) {
-          dec_compute_one<NB, SINGLE, true>(st[4 * r + de], dm, lut_lane, xv, bm_e);
-#pragma unroll
-          for (int i = 0; i < kDecTG; ++i) sr_e[i] = st[4 * r + de].s[i].x;
-          if (de + 4 * kQ < hi)
-            dec_load_w<NB, SINGLE>(st[4 * r + de], wq + (4 * kQ + de) * kUnitBytes, sq + (4 * kQ + de) * kUnitBytes);
-        } else {  // the range starts at the odd chunk
-#pragma unroll
-          for (int i = 0; i < kDecTG; ++i) {
-            sr_e[i] = 0u;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dm[i][e] = 0.f;
-          }
-        }
-        if (dd >= lo && dd < hi) {
-          dec_compute_one<NB, SINGLE, false>(st[4 * r + dd], dm, lut_lane, xv, bm_o);
-#pragma unroll
-          for (int i = 0; i < kDecTG; ++i) sr_o[i] = st[4 * r + dd].s[i].x;
-          if (dd + 4 * kQ < hi)
-            dec_load_w<NB, SINGLE>(st[4 * r + dd], wq + (4 * kQ + dd) * kUnitBytes, sq + (4 * kQ + dd) * kUnitBytes);
-        } else {  // the range ends at the even chunk
-#pragma unroll
-          for (int i = 0; i < kDecTG; ++i) sr_o[i] = 0u;
-        }
-        scale_pair();
-      }
-      const bool pair_end = cq + 4 == p.C && 4 * q + 4 <= u1;  // the range reaches the pair's last chunk
-      if (pair_end || q == q_end - 1) {
-        close_pair(pair_end ? p.C - 1 : (u1 - 1) - cur_pair * p.C);
-        dec_zero<NB>(acc);
-        ++cur_pair;
-        c_first = 0;
-        cq = 0;
-      } else {
-        cq += 4;
-      }
-    };
-    for (int q = q0 - q0 % kQ; q < q_end; q += kQ) {
-      quad(std::integral_constant<int, 0>{}, q);
-      if constexpr (kQ > 1) quad(std::integral_constant<int, 1>{}, q + 1);
-    }
-  } else {
   int ub = 0;
   // Full rounds: every stage computes and refills.
   for (; ub + 2 * D <= n_units; ub += D) {
@@ -924,7 +524,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     }
   }
   if (n_units > 0 && cur_c != 0) close_pair(cur_c - 1);
-  }
   __syncthreads();
 
   // ---- level 2: pairs split between warps, reduced by one warp of the CTA
@@ -947,10 +546,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
     // before it and only its last one ends after it
     const int cf = pr == pair_lo ? cta_first : int(blockIdx.x);
     const int cl = pr == pair_hi ? cta_last : int(blockIdx.x);
-    if constexpr (SINGLE) {
-      dec_reduce_one(p, pr, q0, q1, v0, v1, cf, cl, wb, parts, part_bytes, lane, ep);
-      continue;
-    }
     // the contributors' partials, added in warp order (all loads independent)
     dec_zero<NB>(acc);
 #pragma unroll
@@ -1025,12 +620,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   }
 }
 
-template <int NB, int D, bool SINGLE, bool FUSED = false>
-__global__ void __launch_bounds__(dec_warps(SINGLE) * 32, 1) decode_kernel(const DecodeParams p) {
+template <int NB, int D>
+__global__ void __launch_bounds__(dec_warps(false) * 32, 1) decode_kernel(const DecodeParams p) {
   // The next kernel may launch now: it streams its own weights and waits for
   // this grid's completion before it touches anything this grid writes.
   pdl_launch_dependents();
-  decode_body<NB, D, SINGLE, FUSED>(p, DecWaitPdl{});
+  decode_body<NB, D>(p, DecWaitPdl{});
 }
 
 }  // namespace w4a8

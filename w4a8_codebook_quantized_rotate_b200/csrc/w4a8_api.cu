@@ -83,8 +83,8 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(decode_one_kernel<false>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_one_kernel<true>, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_chain_kernel, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
-          allow_smem(decode_kernel<1, kDecDepth1, false>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
-          allow_smem(decode_kernel<2, kDecDepth2, false>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<1, kDecDepth1>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<2, kDecDepth2>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess ||
           allow_smem(gemm_sk_kernel, 232448) != cudaSuccess)  // the largest sk_smem_bytes over token tiles
         return W4A8_ERR_CUDA;
@@ -102,7 +102,7 @@ w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK
 
 // One token runs the one-token decode kernel, 2..64 tokens the mma.sync
 // decode kernel in slices of up to 16 tokens, more the prefill GEMM -- except
-// that 64..256 tokens on a layer with few 128-row tiles (the GEMM would leave
+// that 64..128 tokens on a layer with few 128-row tiles (the GEMM would leave
 // most SMs idle: 40 CTAs at N = 5120) run the small-batch tensor-core kernel,
 // which splits the weight stream over every SM.
 constexpr int kDecodeSliceM = 16;
@@ -112,6 +112,7 @@ constexpr int kDecodeMaxM = 64;
 #endif
 constexpr int64_t kSkMinM = W4A8_SK_MIN_M;
 constexpr int64_t kSkMaxRowTiles = 100;  // more 128-row tiles than this keep the GEMM busy enough
+constexpr int64_t kSkMaxM = 128;         // measured: ahead of the GEMM at 64 and 128 tokens, behind at 256
 
 static_assert(size_t(kSkMaxCtas) * 8 * 4 <= kWsXchBytes, "the small-batch counters fit in the zero region");
 
@@ -129,7 +130,7 @@ struct LinearPlan {
 
 LinearPlan linear_plan(int64_t M, int64_t K, int64_t N, bool allow_sk = true) {
   LinearPlan L{};
-  L.sk = allow_sk && M >= kSkMinM && M <= kSkMaxTokens && (N + kSkRows - 1) / kSkRows < kSkMaxRowTiles;
+  L.sk = allow_sk && M >= kSkMinM && M <= kSkMaxM && (N + kSkRows - 1) / kSkRows < kSkMaxRowTiles;
   L.decode = !L.sk && M <= kDecodeMaxM;
   L.T = int(N / kTileRows);
   L.C = int(K / kChunkK);
@@ -371,9 +372,9 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     else if (ms == 1)
       e = launch_pdl(decode_one_kernel<false>, grid, dim3(kOneThreads), smem, s, p);
     else if (nb == 1)
-      e = launch_pdl(decode_kernel<1, kDecDepth1, false>, grid, dim3(wpc * 32), smem, s, p);
+      e = launch_pdl(decode_kernel<1, kDecDepth1>, grid, dim3(wpc * 32), smem, s, p);
     else
-      e = launch_pdl(decode_kernel<2, kDecDepth2, false>, grid, dim3(wpc * 32), smem, s, p);
+      e = launch_pdl(decode_kernel<2, kDecDepth2>, grid, dim3(wpc * 32), smem, s, p);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
   }
   return W4A8_OK;
