@@ -30,15 +30,19 @@ namespace w4a8 {
 constexpr int kTcRows = 128;      // weight rows per tile (TMEM lanes, MMA M)
 constexpr int kTcTokens = 256;    // tokens per tile (MMA N)
 constexpr int kTcBK = 64;         // k per pipeline stage
-constexpr int kTcStagesB = 3;     // x_q stages in shared memory
-constexpr int kTcStagesA = 4;     // expanded-weight stages in TMEM
+// Pipeline stages: an x_q tile in shared memory + an expanded-weight tile in
+// TMEM.  Three lie above the table; a fourth goes in the table's alignment
+// room when that room holds it (it does for a kernel without static shared
+// memory; the kernel checks), so 128 KB of activation tiles are in flight.
+constexpr int kTcStages = 4;
+constexpr int kTcStagesHigh = 3;
 constexpr int kTcThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 expansion + epilogue (2 groups)
 constexpr uint32_t kTcStageBBytes = kTcTokens * kTcBK * 2;  // 32 KiB
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcAccCol = 0;     // accumulator: columns [0, 256)
 constexpr uint32_t kTcACol = 256;     // A stages: columns [256, 384)
 // dynamic shared memory: [barriers | pad to the next 64 KiB boundary] [LUT 64 KiB] [B stages]
-constexpr size_t kTcSmemBytes = 1024 + 65536 + 65536 + size_t(kTcStagesB) * kTcStageBBytes;
+constexpr size_t kTcSmemBytes = 1024 + 65536 + 65536 + size_t(kTcStagesHigh) * kTcStageBBytes;
 
 struct TcParams {
   const uint8_t* units;   // unit region of the packed layer
@@ -50,11 +54,16 @@ struct TcParams {
   int M, N, K, C, T;
 };
 
+// One barrier pair per stage: `full` completes when the stage's x_q tile has
+// landed (the TMA thread's arrive with the transfer bytes) and its weight
+// tile is in TMEM (128 expansion threads' arrivals); `empty` when the MMAs
+// that read both have completed.  The MMA thread then waits once and
+// commits once per 64-k block: its per-block work is what bounds the
+// pipeline (measured: two waits and two commits per block held the tensor
+// pipe at 45 %).
 struct TcShared {
-  uint64_t b_full[kTcStagesB];
-  uint64_t b_empty[kTcStagesB];
-  uint64_t a_full[kTcStagesA];
-  uint64_t a_empty[kTcStagesA];
+  uint64_t full[kTcStages];
+  uint64_t empty[kTcStages];
   uint64_t acc_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -147,19 +156,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // 64 KiB aligned (bits 8..15 zero), past the barrier block
   const uint32_t lut = (base + uint32_t(sizeof(TcShared)) + 0xFFFFu) & ~0xFFFFu;
   const uint32_t bstage0 = lut + 65536u;  // 1024-byte aligned
+  // stage 3 in the room below the table, if it fits there
+  const uint32_t low_stage = (base + uint32_t(sizeof(TcShared)) + 1023u) & ~1023u;
+  const int S = low_stage + kTcStageBBytes <= lut ? kTcStages : kTcStagesHigh;
+  auto bstage = [&](int st) { return st < kTcStagesHigh ? bstage0 + uint32_t(st) * kTcStageBBytes : low_stage; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcRows;
   const int m0 = blockIdx.y * kTcTokens;
   const int KB = p.C;  // k blocks of 64
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStagesB; ++s) {
-      mbar_init(&sh->b_full[s], 1);
-      mbar_init(&sh->b_empty[s], 1);
-    }
-    for (int s = 0; s < kTcStagesA; ++s) {
-      mbar_init(&sh->a_full[s], 128);
-      mbar_init(&sh->a_empty[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&sh->full[s], 129);  // 128 expansion threads + the TMA thread
+      mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->acc_full, 1);
     mbar_init(&sh->drain, 1);
@@ -192,37 +201,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmap_x);
       pdl_wait();  // x_q and s_x are written by the previous kernel
-      int issued = 0;
+      int issued = 0, s = 0;
+      uint32_t phase = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % kTcStagesB;
-        if (!tc_wait(&sh->b_empty[s], ((kb / kTcStagesB) & 1) ^ 1, sh, p.err)) break;
-        mbar_arrive_expect_tx(&sh->b_full[s], kTcStageBBytes);
-        tma_load_2d(bstage0 + uint32_t(s) * kTcStageBBytes, &tmap_x, &sh->b_full[s], kb * kTcBK, m0);
+        if (!tc_wait(&sh->empty[s], phase ^ 1u, sh, p.err)) break;
+        mbar_arrive_expect_tx(&sh->full[s], kTcStageBBytes);
+        tma_load_2d(bstage(s), &tmap_x, &sh->full[s], kb * kTcBK, m0);
         ++issued;
+        if (++s == S) {
+          s = 0;
+          phase ^= 1u;
+        }
       }
-      if (sh->abort) {  // let copies already in flight land before the CTA exits
-        for (int i = issued > kTcStagesB ? issued - kTcStagesB : 0; i < issued; ++i)
-          mbar_wait_bounded(&sh->b_full[i % kTcStagesB], (i / kTcStagesB) & 1, p.err, 1u << 20);
+      if (sh->abort && issued > 0) {
+        // The stage barriers also count the expansion threads, which may have
+        // stopped: let the copies in flight land by waiting a fixed, bounded
+        // time (a 32 KB tile lands in microseconds) before the CTA exits.
+        unsigned long long t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        do {
+          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        } while (t - t0 < 50000ull);  // 50 us
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
+      // descriptor of stage 0's first k16 step; a stage adds kTcStageBBytes and a
+      // k16 step 32 bytes to the address field (in 16-byte units; no carry:
+      // the stages lie below 256 KiB)
+      const uint64_t bd_first = sw128_desc(bstage0), bd_low = sw128_desc(low_stage);
+      int s = 0;
+      uint32_t phase = 0;
       for (int kb = 0; kb < KB && ok; ++kb) {
-        const int sa = kb % kTcStagesA, sb = kb % kTcStagesB;
-        ok = tc_wait(&sh->a_full[sa], (kb / kTcStagesA) & 1, sh, p.err) &&
-             tc_wait(&sh->b_full[sb], (kb / kTcStagesB) & 1, sh, p.err);
+        ok = tc_wait(&sh->full[s], phase, sh, p.err);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t a0 = tmem + kTcACol + uint32_t(s) * 32u;
 #pragma unroll
-        for (int j = 0; j < kTcBK / 16; ++j) {
-          const uint32_t a = tmem + kTcACol + uint32_t(sa) * 32u + uint32_t(j) * 8u;
-          const uint64_t bd = sw128_desc(bstage0 + uint32_t(sb) * kTcStageBBytes + uint32_t(j) * 32u);
-          tc_mma_ts_f16(tmem + kTcAccCol, a, bd, kTcIdesc, (kb | j) != 0 ? 1u : 0u);
+        for (int j = 0; j < kTcBK / 16; ++j)
+          tc_mma_ts_f16(tmem + kTcAccCol, a0 + uint32_t(j) * 8u,
+                        (s < kTcStagesHigh ? bd_first + uint64_t(s) * (kTcStageBBytes >> 4) : bd_low) + uint64_t(2 * j),
+                        kTcIdesc,
+                        (kb | j) != 0 ? 1u : 0u);
+        tc_commit(&sh->empty[s]);
+        if (++s == S) {
+          s = 0;
+          phase ^= 1u;
         }
-        tc_commit(&sh->a_empty[sa]);
-        tc_commit(&sh->b_empty[sb]);
       }
       if (ok) {
         tc_commit(&sh->acc_full);
@@ -254,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = 0; i < PF; ++i) {
         const int kb = kb0 + 2 * i;
         if (kb < KB && ok) {
-          const int sa = kb % kTcStagesA;
+          const int sa = kb % S;
           uint32_t v[32];
           exp_compute(es[i], lut_lane, h, v);
           if (!valid) {
@@ -264,14 +291,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           exp_load(es[i], p, tile, kb + 2 * PF, g, valid);
           // lane 0 polls; the outcome is made warp-uniform before the
           // .sync.aligned TMEM store
-          int w_ok = lane == 0 ? int(tc_wait(&sh->a_empty[sa], ((kb / kTcStagesA) & 1) ^ 1, sh, p.err)) : 0;
+          int w_ok = lane == 0 ? int(tc_wait(&sh->empty[sa], ((kb / S) & 1) ^ 1, sh, p.err)) : 0;
           ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
           if (ok) {
             tc_fence_after();
             tmem_st_32x32b_x32(tmem + trow + kTcACol + uint32_t(sa) * 32u, v);
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&sh->a_full[sa]);
+            mbar_arrive(&sh->full[sa]);
           }
         }
       }
