@@ -156,6 +156,34 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * w4a8_linear for an input that another engine delivers (ConvRot card, "Why
+ * this exists": a decode step is bound by streaming memory, so its host
+ * transfers should overlap the previous layer).  Instead of a stream
+ * dependency on the copy that brings x, the call's first kernel waits on the
+ * GPU until x_ready[0] != 0, and once every CTA of that kernel has seen it,
+ * clears x_ready[0] and x_ready[1] (an arrival count).  The caller copies x
+ * and then writes a non-zero word to x_ready[0] (for example a second
+ * cudaMemcpyAsync on the copy stream, which orders it after the data), and
+ * orders its next write of the same x, x_ready and y after this call
+ * (events on the compute stream).  A compute stream holding only kernels
+ * keeps the overlap of consecutive layers (programmatic dependent launch);
+ * a kernel that also waits on a copy event loses it (measured: 18.5 vs
+ * 14.2 us per one-token step).
+ *   x_ready  device, 2 words, 8-byte aligned, [1] zero before the first call;
+ *            a buffer set per call in flight.  The wait is bounded (about a
+ *            second); if it runs out, w4a8_get_device_error reports
+ *            W4A8_ERR_TIMEOUT and the output is undefined.
+ * For one token the layer's single kernel waits (before its wait for the
+ * previous kernel, so the two overlap); otherwise a one-thread kernel waits
+ * and then w4a8_linear_prepare and w4a8_linear_run follow.
+ * Other arguments and errors as w4a8_linear.
+ */
+w4a8_status w4a8_linear_flagged(const uint16_t* x, int64_t M, int64_t K,
+                                const void* packed, int64_t N, uint16_t* y,
+                                unsigned* x_ready, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * The two halves of w4a8_linear, for callers that apply several layers of
  * the same shape to one activation or that time the GEMM on its own.
  *

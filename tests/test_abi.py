@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
         "w4a8_chain_plan", "w4a8_chain_plan_bytes", "w4a8_chain_run", "w4a8_chain_workspace_bytes",
         "w4a8_compare", "w4a8_compare_workspace_bytes", "w4a8_convert_weight", "w4a8_convert_workspace_bytes",
         "w4a8_decode_chain", "w4a8_decode_chain_workspace_bytes", "w4a8_dense_reference",
-        "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_prepare",
+        "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_flagged",
+        "w4a8_linear_prepare",
         "w4a8_linear_run",
         "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
         "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_selftest_timeout", "w4a8_status_string",

@@ -1,0 +1,78 @@
+"""GPU tests of w4a8_linear_flagged: the layer waits on the GPU for a ready
+word that the caller's copy writes after x, instead of a stream dependency
+on that copy (which would cost the overlap of consecutive layers)."""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(lib, n, k, seed):
+    q = synth.quantized_format(n, k, synth.rng_for(60, seed, "qfmt"))
+    t = {kk: torch.from_numpy(np.ascontiguousarray(v)).cuda() for kk, v in q.items()}
+    return lib.pack_layout(t["packed"], t["s_rel"], t["s_ch"], t["cb"])
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 5120, 1024), (1, 9216, 512), (4, 768, 592), (100, 512, 256)])
+def test_flagged_equals_linear_and_clears_its_flag(lib, m, k, n):
+    packed = _layer(lib, n, k, k + m)
+    x = torch.randn((m, k), device="cuda").to(torch.bfloat16)
+    ref = lib.linear(x, packed, n)
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    ready = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        ready[0] = 1
+        lib.linear_flagged(x, packed, n, ready, ws, y)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+        assert ready.tolist() == [0, 0]  # cleared for the caller's next copy
+    assert lib.get_device_error() == 0
+
+
+def test_flagged_input_from_a_copy_on_another_stream(lib):
+    """x and its ready word arrive by copies on a second stream; the layer's
+    stream never waits on that stream's events."""
+    m, k, n = 1, 5120, 2048
+    packed = _layer(lib, n, k, 7)
+    x_host = torch.randn((m, k)).to(torch.bfloat16).pin_memory()
+    one = torch.tensor([1, 0], dtype=torch.int32).pin_memory()
+    ref = lib.linear(x_host.cuda(), packed, n)
+    x_dev = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
+    ready = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    copy = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    lib.linear_flagged(x_dev, packed, n, ready, ws, y)     # launched first: waits on the GPU
+    with torch.cuda.stream(copy):
+        x_dev.copy_(x_host, non_blocking=True)
+        ready[:1].copy_(one[:1], non_blocking=True)          # after the data, same stream
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    assert ready.tolist() == [0, 0]
+    assert lib.get_device_error() == 0
+
+
+def test_flagged_wait_runs_out_and_reports_a_timeout(lib):
+    """A ready word nothing sets: the bounded wait gives up (about a second),
+    the call records a timeout, and the context stays usable."""
+    m, k, n = 1, 512, 256
+    packed = _layer(lib, n, k, 9)
+    x = torch.randn((m, k), device="cuda").to(torch.bfloat16)
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    ready = torch.zeros(2, dtype=torch.int32, device="cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    lib.linear_flagged(x, packed, n, ready, ws, y)
+    assert lib.get_device_error() == 6  # W4A8_ERR_TIMEOUT, read and cleared
+    ready.zero_()
+    ws.zero_()  # the workspace after a timeout, as the header asks
+    ready[0] = 1
+    lib.linear_flagged(x, packed, n, ready, ws, y)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), lib.linear(x, packed, n).view(torch.int16))
+    assert lib.get_device_error() == 0

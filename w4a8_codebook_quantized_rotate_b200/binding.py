@@ -28,7 +28,7 @@ EXPORTS = (
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
     "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
-    "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain",
+    "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain", "w4a8_linear_flagged",
 )
 
 
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_chain_run": (st, [vp, i64, vp, sz, vp]),
         "w4a8_decode_chain_workspace_bytes": (sz, [vp, i64]),
         "w4a8_decode_chain": (st, [vp, i64, vp, sz, vp]),
+        "w4a8_linear_flagged": (st, [vp, i64, i64, vp, i64, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -417,3 +418,21 @@ class DecodeChain:
     def run(self, stream=None) -> None:
         _check("w4a8_decode_chain", load_library().w4a8_decode_chain(
             self._arr, self.n_layers, self.workspace.data_ptr(), self.workspace.numel(), _stream(stream)))
+
+
+def linear_flagged(x: torch.Tensor, packed: torch.Tensor, n: int, x_ready: torch.Tensor,
+                   workspace: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """w4a8_linear that waits on the GPU for ``x_ready[0] != 0`` (an int32
+    CUDA tensor of 2 words written by the caller's copy after x) instead of a
+    stream dependency; the layer clears the flag once it has read x."""
+    lib = load_library()
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(packed, torch.uint8, "packed")
+    _cuda(x_ready, torch.int32, "x_ready")
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(out, torch.bfloat16, "out")
+    m, k = x.shape
+    _check("w4a8_linear_flagged", lib.w4a8_linear_flagged(
+        x.data_ptr(), m, k, packed.data_ptr(), n, out.data_ptr(), x_ready.data_ptr(), workspace.data_ptr(),
+        workspace.numel(), _stream(stream)))
+    return out

@@ -98,6 +98,10 @@ struct DecodeParams {
   const unsigned* in_amax;
   unsigned* zero_cnt;
   int zero_n;
+  // One token, input from another engine (w4a8_linear_flagged): every CTA
+  // waits until x_ready[0] != 0 before reading x; the last CTA to see it
+  // clears x_ready[0] and x_ready[1] (its arrival count).  Null: no wait.
+  unsigned* x_ready;
 };
 
 // Floats of one partial (a tile pair, the first M tokens).

@@ -427,6 +427,18 @@ __device__ __forceinline__ void decode_one_body(const DecodeParams& p, const Wai
                    "r"(*reinterpret_cast<const uint32_t*>(&h)));
     }
   };
+  if (p.x_ready) {
+    // x comes from another engine: wait (bounded) for its ready word, which
+    // no earlier kernel touches, so this overlaps the previous kernel
+    if (threadIdx.x == 0) {
+      poll_at_least_bounded(p.x_ready, 1u, p.err, 1u << 21);  // about a second
+      if (atomicAdd(p.x_ready + 1, 1u) == gridDim.x - 1) {  // the last CTA to see it clears it
+        p.x_ready[0] = 0u;
+        p.x_ready[1] = 0u;
+      }
+    }
+    __syncthreads();  // the CTA reads x after thread 0's acquire
+  }
   wait_inputs();  // x (or the prepared codes) and the workspace come from an earlier step
   if (p.zero_cnt && blockIdx.x == 0)
     for (int i = threadIdx.x; i < p.zero_n; i += kOneThreads) p.zero_cnt[i] = 0u;

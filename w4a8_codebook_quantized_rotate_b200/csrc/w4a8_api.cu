@@ -217,6 +217,17 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 
 }  // namespace
 
+// Waits (bounded) until ready[0] != 0, clears ready[0] and ready[1], then
+// waits for the previous kernel (so that the next kernel's wait covers it
+// too).  One thread.
+__global__ void flag_wait_kernel(unsigned* ready, unsigned* err) {
+  pdl_launch_dependents();
+  poll_at_least_bounded(ready, 1u, err, 1u << 21);  // about a second
+  ready[0] = 0u;
+  ready[1] = 0u;
+  pdl_wait();
+}
+
 // A word nothing ever writes: the self-test's flag.
 __device__ unsigned g_never_set;
 
@@ -330,7 +341,8 @@ static void one_token_split(DecodeParams& p, int ctas_avail) {
 // and quantises the token; otherwise it reads what w4a8_linear_prepare left
 // in the workspace.
 static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, int64_t M, int64_t K, int64_t N,
-                                 const uint8_t* pk, uint16_t* y, uint8_t* ws, cudaStream_t s, const uint16_t* x) {
+                                 const uint8_t* pk, uint16_t* y, uint8_t* ws, cudaStream_t s, const uint16_t* x,
+                                 unsigned* x_ready = nullptr) {
   const PackedLayout L = packed_layout(N, K);
   for (int sl = 0; sl < plan.slices; ++sl) {
     const int64_t m0 = int64_t(sl) * kDecodeSliceM;
@@ -347,6 +359,7 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     p.xch = reinterpret_cast<unsigned long long*>(ws);
     p.counters = reinterpret_cast<unsigned*>(ws + kWsCntOff);
     p.err = d->err;
+    p.x_ready = x_ready;
     p.M = int(ms);
     p.N = int(N);
     p.K = int(K);
@@ -496,6 +509,24 @@ w4a8_status w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const void* pac
     return launch_decode(plan, d, M, K, N, static_cast<const uint8_t*>(packed), y, static_cast<uint8_t*>(workspace),
                          static_cast<cudaStream_t>(stream), x);
   }
+  w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
+  if (st != W4A8_OK) return st;
+  return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_linear_flagged(const uint16_t* x, int64_t M, int64_t K, const void* packed, int64_t N, uint16_t* y,
+                                unsigned* x_ready, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !packed || !y || !workspace || !x_ready) return W4A8_ERR_NULL;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (reinterpret_cast<uintptr_t>(x_ready) & 7u))
+    return W4A8_ERR_ALIGN;
+  LinearPlan plan;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = linear_checks(M, K, N, workspace, workspace_bytes, &plan, &d); st != W4A8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 1)  // the layer's single kernel waits for the flag itself
+    return launch_decode(plan, d, M, K, N, static_cast<const uint8_t*>(packed), y, static_cast<uint8_t*>(workspace), s,
+                         x, x_ready);
+  if (launch_pdl(flag_wait_kernel, dim3(1), dim3(1), 0, s, x_ready, d->err) != cudaSuccess) return W4A8_ERR_CUDA;
   w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
