@@ -15,6 +15,10 @@ Sources (page title and section):
   and "Reproducing" -- called the *ConvRot card* below.
 * "Qwen3.8-27B-W4A8" model card (CuTIsolation), sections "Model Overview" and
   "Accuracy" -- called the *W4A8 card* below.
+* "Qwen3.8-27B-Uncensored-NVFP4: En runbook för servering på Blackwell-GPU:er",
+  section "Vad NVFP4 är, och hur det skiljer sig från FP8 och från INT8/AWQ"
+  -- the *NVFP4 runbook*: the format of the comparison foil in
+  :mod:`oracle.nvfp4_ref` (imported explicitly, not re-exported here).
 
 Every function in :mod:`oracle.w4a8_ref` names the passage it follows.  Where
 the pages leave a step open, the reading taken is written beside the code.
