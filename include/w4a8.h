@@ -374,6 +374,82 @@ w4a8_status w4a8_compare(const void* a, int32_t a_is_bf16, const float* ref, int
 w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const float* w,
                                  int64_t N, float* y, void* stream);
 
+/* ------------------------------------------------------------------------
+ * NVFP4 comparison layer (the speed and accuracy foil of the codebook layer)
+ *
+ * Format: "Qwen3.8-27B-Uncensored-NVFP4: En runbook för servering på
+ * Blackwell-GPU:er", section "Vad NVFP4 är, och hur det skiljer sig från FP8
+ * och från INT8/AWQ": E2M1 values (1 sign, 2 exponent, 1 mantissa bit), one
+ * e4m3 scale per 16 values, one fp32 scalar per tensor; Blackwell runs the
+ * FP4 matmul natively.  Both operands are 4-bit here (the native block-scaled
+ * FP4 tensor-core instruction takes FP4 on both sides).  Readings taken where
+ * the page is silent: E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; round to
+ * nearest even, saturating; g = amax / (6 * 448); weights one g per tensor,
+ * activations one g per token; both operands rotated like the codebook layer
+ * (each 256-block of K times H_256 / 16).  In fp32: d = g * 6, block scale
+ * s = e4m3(bmax / d), S = value(s) * g, code = e2m1(x / S) (0 where S = 0).
+ *
+ * Layouts (all device memory, caller-owned):
+ *   codes   uint8 [R, K/2]: two codes per byte, even k in the low nibble.
+ *   scales  uint8 e4m3 codes in the tensor cores' order, rows padded to a
+ *           multiple of 128 (w4a8_nvfp4_scale_bytes): 512-byte chunks of 128
+ *           rows x 64 k in [row block][k/64] order; inside a chunk the scale
+ *           of (row r, 16-block c) is byte 16 (r % 32) + 4 ((r % 128) / 32)
+ *           + c % 4.  Pad rows hold 0.
+ *   g       fp32 [R].
+ * Shapes: R, M, N in [1, 2^24]; K a multiple of 256, at most W4A8_MAX_K.
+ * Pointers 16-byte aligned.  Calls are asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of a scale buffer for R rows of K values (0 for a bad shape). */
+size_t w4a8_nvfp4_scale_bytes(int64_t R, int64_t K);
+
+/*
+ * Quantise R rows of x [R, K] (bf16 bits when x_is_f32 == 0, else fp32) to
+ * NVFP4: codes, scales (tensor-core order) and g.  rotate != 0 rotates each
+ * row first.  per_tensor != 0 takes one g for the whole tensor (weights; it
+ * then needs `amax_scratch`, one device word the call overwrites); else one g
+ * per row (activations; `amax_scratch` may be NULL).
+ * Errors: NULL, SHAPE, ALIGN, ARCH, CUDA.
+ */
+w4a8_status w4a8_nvfp4_quantize(const void* x, int32_t x_is_f32, int64_t R, int64_t K,
+                                int32_t rotate, int32_t per_tensor, uint8_t* codes,
+                                uint8_t* scales, float* g, unsigned* amax_scratch,
+                                void* stream);
+
+/*
+ * Row-major e4m3 scale codes [R, K/16] -> the tensor-core order
+ * (w4a8_nvfp4_scale_bytes(R, K) bytes; pad rows 0).  For scales made
+ * elsewhere.  Errors: NULL, SHAPE, ARCH, CUDA.
+ */
+w4a8_status w4a8_nvfp4_pack_scales(const uint8_t* scales_rows, int64_t R, int64_t K,
+                                   uint8_t* scales, void* stream);
+
+/*
+ * y [M, N] (bf16 bits) = g_x[m] g_w[n] sum_k (e2m1 x e4m3)(x)[m, k]
+ * (e2m1 x e4m3)(w)[n, k], on the block-scaled FP4 tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, fp32 accumulation).  x_codes [M, K/2],
+ * x_scales, g_x [M]; w_codes [N, K/2], w_scales, g_w [N].  A bounded wait
+ * that gives up leaves y undefined and is reported by w4a8_get_device_error.
+ * Errors: NULL, SHAPE, ALIGN, ARCH, CUDA.
+ */
+w4a8_status w4a8_nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* g_x,
+                            int64_t M, const uint8_t* w_codes, const uint8_t* w_scales,
+                            const float* g_w, int64_t N, int64_t K, uint16_t* y, void* stream);
+
+/* Workspace bytes of w4a8_nvfp4_linear for M tokens of K values. */
+size_t w4a8_nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The NVFP4 layer: rotate and quantise x [M, K] (bf16 bits, one g per token)
+ * into `workspace`, then w4a8_nvfp4_gemm against weights quantised with
+ * rotate != 0.  Errors: as the two calls, WORKSPACE if the workspace is
+ * smaller than w4a8_nvfp4_linear_workspace_bytes.
+ */
+w4a8_status w4a8_nvfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* w_codes,
+                              const uint8_t* w_scales, const float* g_w, int64_t N, uint16_t* y,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Synchronise `stream`, then report and clear the device-side error word of
  * the current device: W4A8_ERR_TIMEOUT if a bounded wait inside a kernel

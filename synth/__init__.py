@@ -88,6 +88,17 @@ def quantized_format(n: int, k: int, rng: np.random.Generator) -> dict:
     }
 
 
+def nvfp4_operands(rows: int, k: int, rng: np.random.Generator) -> dict:
+    """NVFP4-format operands drawn directly: packed codes [rows, k/2] uint8
+    (every byte value), e4m3 scale codes [rows, k/16] uint8 in 0x20..0x58
+    (the values 1/8 .. 16), fp32 scalars [rows] in [1e-3, 1e-2]."""
+    return {
+        "codes": rng.integers(0, 256, size=(rows, k // 2), dtype=np.uint8),
+        "scales": rng.integers(0x20, 0x59, size=(rows, k // 16), dtype=np.uint8),
+        "g": rng.uniform(1e-3, 1e-2, size=rows).astype(np.float32),
+    }
+
+
 def quantized_format_device(n: int, k: int, seed: int, device):
     """Same distributions as :func:`quantized_format`, drawn by torch's
     generator directly on ``device`` (for multi-GB throughput inputs)."""

@@ -33,7 +33,9 @@ def test_header_declares_the_boundary():
         "w4a8_get_device_error", "w4a8_linear", "w4a8_linear_decode_static", "w4a8_linear_flagged",
         "w4a8_linear_prepare",
         "w4a8_linear_run",
-        "w4a8_linear_workspace_bytes", "w4a8_pack_layout",
+        "w4a8_linear_workspace_bytes", "w4a8_nvfp4_gemm", "w4a8_nvfp4_linear",
+        "w4a8_nvfp4_linear_workspace_bytes", "w4a8_nvfp4_pack_scales", "w4a8_nvfp4_quantize",
+        "w4a8_nvfp4_scale_bytes", "w4a8_pack_layout",
         "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_selftest_timeout", "w4a8_status_string",
         "w4a8_unpack_dequant"])
 
@@ -60,6 +62,31 @@ def test_packed_bytes_layout_arithmetic(lib):
 def test_bad_weight_shapes_have_zero_size(lib, n, k):
     assert lib.w4a8_packed_bytes(n, k) == 0
     assert lib.w4a8_linear_workspace_bytes(1, k, n) == 0
+
+
+def test_nvfp4_sizes(lib):
+    """Scales: rows padded to 128, one byte per 16 values; the layer's
+    workspace holds the activation codes, scales and per-token scalars."""
+    assert lib.w4a8_nvfp4_scale_bytes(17408, 5120) == 17408 * 5120 // 16
+    assert lib.w4a8_nvfp4_scale_bytes(1, 256) == 128 * 16
+    assert lib.w4a8_nvfp4_scale_bytes(129, 512) == 256 * 32
+    for r, k in ((0, 256), (1, 128), (1, 300), (1, 65536), (-1, 256)):
+        assert lib.w4a8_nvfp4_scale_bytes(r, k) == 0
+        assert lib.w4a8_nvfp4_linear_workspace_bytes(r, k) == 0
+    ws = lib.w4a8_nvfp4_linear_workspace_bytes(4096, 5120)
+    assert ws >= 4096 * 5120 // 2 + 4096 * 5120 // 16 + 4096 * 4
+
+
+def test_nvfp4_refuses_bad_arguments_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(4096)
+    assert lib.w4a8_nvfp4_gemm(None, fake, fake, 16, fake, fake, fake, 128, 256, fake, None) == 1
+    assert lib.w4a8_nvfp4_gemm(fake, fake, fake, 16, fake, fake, fake, 128, 200, fake, None) == 2
+    assert lib.w4a8_nvfp4_gemm(fake, fake, fake, 0, fake, fake, fake, 128, 256, fake, None) == 2
+    assert lib.w4a8_nvfp4_gemm(vp(4097), fake, fake, 16, fake, fake, fake, 128, 256, fake, None) == 3
+    assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 256, 1, 1, fake, fake, fake, None, None) == 1
+    assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 100, 1, 0, fake, fake, fake, None, None) == 2
+    assert lib.w4a8_nvfp4_linear(fake, 4, 256, fake, fake, fake, 128, fake, fake, 16, None) == 4
 
 
 # Every workspace starts with the words that join partial sums across CTAs:

@@ -29,6 +29,8 @@ EXPORTS = (
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
     "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
     "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain", "w4a8_linear_flagged",
+    "w4a8_nvfp4_scale_bytes", "w4a8_nvfp4_quantize", "w4a8_nvfp4_pack_scales", "w4a8_nvfp4_gemm",
+    "w4a8_nvfp4_linear_workspace_bytes", "w4a8_nvfp4_linear",
 )
 
 
@@ -81,6 +83,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_decode_chain_workspace_bytes": (sz, [vp, i64]),
         "w4a8_decode_chain": (st, [vp, i64, vp, sz, vp]),
         "w4a8_linear_flagged": (st, [vp, i64, i64, vp, i64, vp, vp, vp, sz, vp]),
+        "w4a8_nvfp4_scale_bytes": (sz, [i64, i64]),
+        "w4a8_nvfp4_quantize": (st, [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, ctypes.c_int32,
+                                     vp, vp, vp, vp, vp]),
+        "w4a8_nvfp4_pack_scales": (st, [vp, i64, i64, vp, vp]),
+        "w4a8_nvfp4_gemm": (st, [vp, vp, vp, i64, vp, vp, vp, i64, i64, vp, vp]),
+        "w4a8_nvfp4_linear_workspace_bytes": (sz, [i64, i64]),
+        "w4a8_nvfp4_linear": (st, [vp, i64, i64, vp, vp, vp, i64, vp, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -435,4 +444,89 @@ def linear_flagged(x: torch.Tensor, packed: torch.Tensor, n: int, x_ready: torch
     _check("w4a8_linear_flagged", lib.w4a8_linear_flagged(
         x.data_ptr(), m, k, packed.data_ptr(), n, out.data_ptr(), x_ready.data_ptr(), workspace.data_ptr(),
         workspace.numel(), _stream(stream)))
+    return out
+
+
+# ---------------------------------------------------------------- NVFP4 comparison layer
+
+def nvfp4_scale_bytes(rows: int, k: int) -> int:
+    return int(load_library().w4a8_nvfp4_scale_bytes(rows, k))
+
+
+def nvfp4_quantize(x: torch.Tensor, rotate: bool = True, per_tensor: bool = False, stream=None):
+    """x [R, K] (bf16 or fp32) -> (codes uint8 [R, K/2], scales uint8 in the
+    tensor cores' order, g fp32 [R]); one g per tensor or per row."""
+    lib = load_library()
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("x must be bf16 or fp32")
+    _cuda(x, x.dtype, "x")
+    r, k = x.shape
+    nbytes = lib.w4a8_nvfp4_scale_bytes(r, k)
+    if nbytes == 0:
+        raise W4A8Error("w4a8_nvfp4_scale_bytes", 2)
+    codes = torch.empty((r, k // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    g = torch.empty(r, dtype=torch.float32, device=x.device)
+    scratch = torch.empty(4, dtype=torch.int32, device=x.device) if per_tensor else None
+    _check("w4a8_nvfp4_quantize", lib.w4a8_nvfp4_quantize(
+        x.data_ptr(), int(x.dtype == torch.float32), r, k, int(rotate), int(per_tensor), codes.data_ptr(),
+        scales.data_ptr(), g.data_ptr(), scratch.data_ptr() if scratch is not None else None, _stream(stream)))
+    return codes, scales, g
+
+
+def nvfp4_pack_scales(scales_rows: torch.Tensor, stream=None) -> torch.Tensor:
+    """Row-major e4m3 scale codes uint8 [R, K/16] -> the tensor cores' order."""
+    lib = load_library()
+    _cuda(scales_rows, torch.uint8, "scales_rows")
+    r, k = scales_rows.shape[0], scales_rows.shape[1] * 16
+    nbytes = lib.w4a8_nvfp4_scale_bytes(r, k)
+    if nbytes == 0:
+        raise W4A8Error("w4a8_nvfp4_scale_bytes", 2)
+    out = torch.empty(nbytes, dtype=torch.uint8, device=scales_rows.device)
+    _check("w4a8_nvfp4_pack_scales", lib.w4a8_nvfp4_pack_scales(
+        scales_rows.data_ptr(), r, k, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def nvfp4_gemm(x_codes: torch.Tensor, x_scales: torch.Tensor, g_x: torch.Tensor, w_codes: torch.Tensor,
+               w_scales: torch.Tensor, g_w: torch.Tensor, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """y [M, N] bf16 from NVFP4 operands (codes [rows, K/2], scales in the
+    tensor cores' order, g fp32 [rows])."""
+    lib = load_library()
+    for t, name in ((x_codes, "x_codes"), (x_scales, "x_scales"), (w_codes, "w_codes"), (w_scales, "w_scales")):
+        _cuda(t, torch.uint8, name)
+    _cuda(g_x, torch.float32, "g_x")
+    _cuda(g_w, torch.float32, "g_w")
+    m, k = x_codes.shape[0], x_codes.shape[1] * 2
+    n = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != k:
+        raise ValueError("x and w differ in K")
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x_codes.device)
+    _cuda(out, torch.bfloat16, "out")
+    _check("w4a8_nvfp4_gemm", lib.w4a8_nvfp4_gemm(
+        x_codes.data_ptr(), x_scales.data_ptr(), g_x.data_ptr(), m, w_codes.data_ptr(), w_scales.data_ptr(),
+        g_w.data_ptr(), n, k, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def nvfp4_linear(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, g_w: torch.Tensor,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """The NVFP4 layer on bf16 x [M, K] (quantised per token, rotated) against
+    weights from nvfp4_quantize(w, rotate=True, per_tensor=True)."""
+    lib = load_library()
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    n = w_codes.shape[0]
+    if workspace is None:
+        workspace = torch.empty(lib.w4a8_nvfp4_linear_workspace_bytes(m, k), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(out, torch.bfloat16, "out")
+    _check("w4a8_nvfp4_linear", lib.w4a8_nvfp4_linear(
+        x.data_ptr(), m, k, w_codes.data_ptr(), w_scales.data_ptr(), g_w.data_ptr(), n, out.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return out

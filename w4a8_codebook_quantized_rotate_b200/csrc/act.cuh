@@ -65,16 +65,10 @@ __device__ __forceinline__ uint4 load_block_lane(const uint16_t* __restrict__ ro
   return __ldcg(reinterpret_cast<const uint4*>(row + b * kRotBlock + lane * 8));
 }
 
-// Lane's 8 values of a rotated 256-block, from the lane's 16 bytes of it.
-// Three butterfly stages inside the lane, five across lanes (shuffles), then
-// the exact 1/16.
-__device__ __forceinline__ void rotate_words_lane(const uint4 raw, int lane, float (&v)[8]) {
-  const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(wds[i] << 16);
-    v[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
-  }
+// Rotate a 256-block held 8 consecutive values per lane (lane l holds
+// positions 8 l .. 8 l + 7), in place: three butterfly stages inside the
+// lane, five across lanes (shuffles), then the exact 1/16.
+__device__ __forceinline__ void rotate_vals_lane(float (&v)[8], int lane) {
   fwht8_in_lane(v);
 #pragma unroll
   for (int bit = 1; bit < 32; bit <<= 1) {
@@ -87,6 +81,17 @@ __device__ __forceinline__ void rotate_words_lane(const uint4 raw, int lane, flo
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;  // 1/16, exact
+}
+
+// Lane's 8 values of a rotated 256-block, from the lane's 16 bytes of it (bf16).
+__device__ __forceinline__ void rotate_words_lane(const uint4 raw, int lane, float (&v)[8]) {
+  const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(wds[i] << 16);
+    v[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+  }
+  rotate_vals_lane(v, lane);
 }
 
 // Lane's 8 values of the rotated 256-block b of a bf16 row.

@@ -1,6 +1,7 @@
 // C ABI of the W4A8 ConvRot linear layer: argument checks, per-device set-up
 // and kernel launches.  The declarations, with argument meaning, layout,
 // ownership and error behaviour, are in include/w4a8.h.
+#include <algorithm>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -14,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv1.cuh"
+#include "nvfp4.cuh"
 #include "pack.cuh"
 #include "verify.cuh"
 
@@ -86,7 +88,11 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(decode_kernel<1, kDecDepth1>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
           allow_smem(decode_kernel<2, kDecDepth2>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess ||
-          allow_smem(gemm_sk_kernel, 232448) != cudaSuccess)  // the largest sk_smem_bytes over token tiles
+          allow_smem(gemm_sk_kernel, 232448) != cudaSuccess ||  // the largest sk_smem_bytes over token tiles
+          allow_smem(nvfp4_quant_kernel, size_t(kMaxK) * 4) != cudaSuccess ||
+          allow_smem(nvfp4_gemm_kernel<256>, NvCfg<256>::kSmem) != cudaSuccess ||
+          allow_smem(nvfp4_gemm_kernel<128>, NvCfg<128>::kSmem) != cudaSuccess ||
+          allow_smem(nvfp4_gemm_kernel<64>, NvCfg<64>::kSmem) != cudaSuccess)
         return W4A8_ERR_CUDA;
     }
     d.ready = true;
@@ -941,6 +947,149 @@ w4a8_status w4a8_decode_chain(const w4a8_chain_layer* layers, int64_t n_layers, 
 }
 
 // ------------------------------------------------------------------ fidelity checks
+
+// ------------------------------------------------------------------ NVFP4 comparison layer
+
+static bool nv_shape_ok(int64_t R, int64_t K) {
+  return R > 0 && R <= (int64_t(1) << 24) && K > 0 && K % kNvBK == 0 && K <= kMaxK;
+}
+
+size_t w4a8_nvfp4_scale_bytes(int64_t R, int64_t K) { return nv_shape_ok(R, K) ? nv_sf_bytes(R, K) : 0; }
+
+static w4a8_status nv_quantize(const void* x, int32_t x_is_f32, int64_t R, int64_t K, int32_t rotate,
+                               unsigned* amax_word, uint8_t* codes, uint8_t* scales, float* g, cudaStream_t s) {
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  NvQuantParams p;
+  p.x = x;
+  p.amax_word = amax_word;
+  p.codes = codes;
+  p.sf = scales;
+  p.g = g;
+  p.R = int(R);
+  p.K = int(K);
+  p.in_f32 = x_is_f32 ? 1 : 0;
+  p.rotate = rotate ? 1 : 0;
+  if (amax_word) {
+    if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned), s) != cudaSuccess) return W4A8_ERR_CUDA;
+    nvfp4_amax_kernel<<<unsigned(R), kNvQuantThreads, 0, s>>>(p, amax_word);
+    if (launch_status() != W4A8_OK) return W4A8_ERR_CUDA;
+  }
+  const unsigned rows = unsigned((R + 127) / 128 * 128);
+  const cudaError_t e = launch_pdl(nvfp4_quant_kernel, dim3(rows), dim3(kNvQuantThreads), size_t(K) * 4, s, p);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+w4a8_status w4a8_nvfp4_quantize(const void* x, int32_t x_is_f32, int64_t R, int64_t K, int32_t rotate,
+                                int32_t per_tensor, uint8_t* codes, uint8_t* scales, float* g,
+                                unsigned* amax_scratch, void* stream) {
+  if (!x || !codes || !scales || !g || (per_tensor && !amax_scratch)) return W4A8_ERR_NULL;
+  if (!nv_shape_ok(R, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(g)) return W4A8_ERR_ALIGN;
+  return nv_quantize(x, x_is_f32, R, K, rotate, per_tensor ? amax_scratch : nullptr, codes, scales, g,
+                     static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w4a8_nvfp4_pack_scales(const uint8_t* scales_rows, int64_t R, int64_t K, uint8_t* scales,
+                                   void* stream) {
+  if (!scales_rows || !scales) return W4A8_ERR_NULL;
+  if (!nv_shape_ok(R, K)) return W4A8_ERR_SHAPE;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  const int64_t total = int64_t(nv_sf_bytes(R, K));
+  const unsigned blocks = unsigned(std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8));
+  nvfp4_pack_scales_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(scales_rows, int(R), int(K),
+                                                                                  scales);
+  return launch_status();
+}
+
+static w4a8_status nv_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* g_x, int64_t M,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, int64_t N, int64_t K,
+                           uint16_t* y, const DeviceState* d, cudaStream_t s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return W4A8_ERR_CUDA;
+  const int nt = M > 128 ? 256 : M > 64 ? 128 : 64;
+  CUtensorMap tw, tx;
+  const cuuint64_t gw_dim[2] = {cuuint64_t(K / 2), cuuint64_t(N)};
+  const cuuint64_t gx_dim[2] = {cuuint64_t(K / 2), cuuint64_t(M)};
+  const cuuint64_t gstride[1] = {cuuint64_t(K / 2)};
+  const cuuint32_t box_w[2] = {128u, uint32_t(kNvRows)};
+  const cuuint32_t box_x[2] = {128u, uint32_t(nt)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(w_codes), gw_dim, gstride, box_w, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(x_codes), gx_dim, gstride, box_x, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return W4A8_ERR_CUDA;
+  NvGemmParams p;
+  p.sfa = w_scales;
+  p.sfb = x_scales;
+  p.gw = g_w;
+  p.gx = g_x;
+  p.y = y;
+  p.err = d->err;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  const dim3 grid(unsigned((N + kNvRows - 1) / kNvRows), unsigned((M + nt - 1) / nt));
+  cudaError_t e;
+  if (nt == 256)
+    e = launch_pdl(nvfp4_gemm_kernel<256>, grid, dim3(kNvThreads), NvCfg<256>::kSmem, s, tw, tx, p);
+  else if (nt == 128)
+    e = launch_pdl(nvfp4_gemm_kernel<128>, grid, dim3(kNvThreads), NvCfg<128>::kSmem, s, tw, tx, p);
+  else
+    e = launch_pdl(nvfp4_gemm_kernel<64>, grid, dim3(kNvThreads), NvCfg<64>::kSmem, s, tw, tx, p);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+w4a8_status w4a8_nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* g_x, int64_t M,
+                            const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, int64_t N, int64_t K,
+                            uint16_t* y, void* stream) {
+  if (!x_codes || !x_scales || !g_x || !w_codes || !w_scales || !g_w || !y) return W4A8_ERR_NULL;
+  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
+    return W4A8_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  return nv_gemm(x_codes, x_scales, g_x, M, w_codes, w_scales, g_w, N, K, y, d, static_cast<cudaStream_t>(stream));
+}
+
+struct NvLinearWs {
+  size_t off_codes, off_sf, off_g, total;
+};
+static NvLinearWs nv_linear_ws(int64_t M, int64_t K) {
+  NvLinearWs w;
+  w.off_codes = 0;
+  w.off_sf = round_up(size_t(M) * size_t(K / 2), 256);
+  w.off_g = w.off_sf + round_up(nv_sf_bytes(M, K), 256);
+  w.total = w.off_g + round_up(size_t(M) * 4, 256);
+  return w;
+}
+
+size_t w4a8_nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
+  return nv_shape_ok(M, K) ? nv_linear_ws(M, K).total : 0;
+}
+
+w4a8_status w4a8_nvfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* w_codes,
+                              const uint8_t* w_scales, const float* g_w, int64_t N, uint16_t* y, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!x || !w_codes || !w_scales || !g_w || !y || !workspace) return W4A8_ERR_NULL;
+  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace))
+    return W4A8_ERR_ALIGN;
+  const NvLinearWs w = nv_linear_ws(M, K);
+  if (workspace_bytes < w.total) return W4A8_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DeviceState* d = nullptr;
+  if (w4a8_status st = device_state(&d); st != W4A8_OK) return st;
+  float* gx = reinterpret_cast<float*>(ws + w.off_g);
+  if (w4a8_status st = nv_quantize(x, 0, M, K, 1, nullptr, ws + w.off_codes, ws + w.off_sf, gx, s); st != W4A8_OK)
+    return st;
+  return nv_gemm(ws + w.off_codes, ws + w.off_sf, gx, M, w_codes, w_scales, g_w, N, K, y, d, s);
+}
 
 size_t w4a8_compare_workspace_bytes(void) { return size_t(kCmpBlocks) * 3 * sizeof(double); }
 
