@@ -702,14 +702,90 @@ def measure_nvfp4_foil(B, torch, dev, rank, n=17408, k=5120, tokens=16):
         c = B.compare(y, y_ref).cpu()
         out[name] = {"forward_rel_l2": float((c[0] / c[1]).sqrt()), "codebook": [round(float(v), 5) for v in q["cb"]]}
         del q, pk, y
+    # the native NVFP4 layer: 4-bit activations too (one fp32 scalar per token), with and without the rotation
+    wc, wsf, gw = B.nvfp4_quantize(w, rotate=True, per_tensor=True)
+    c = B.compare(B.nvfp4_linear(x, wc, wsf, gw), y_ref).cpu()
+    out["nvfp4_w4a4_rotated"] = {"forward_rel_l2": float((c[0] / c[1]).sqrt())}
+    wc, wsf, gw = B.nvfp4_quantize(w, rotate=False, per_tensor=True)
+    xc, xs, gx = B.nvfp4_quantize(x, rotate=False)
+    c = B.compare(B.nvfp4_gemm(xc, xs, gx, wc, wsf, gw), y_ref).cpu()
+    out["nvfp4_w4a4_unrotated"] = {"forward_rel_l2": float((c[0] / c[1]).sqrt())}
+    del wc, wsf, gw, xc, xs, gx
     del w, x, y_ref
     torch.cuda.empty_cache()
     return {"workload": f"W [{n}, {k}] ~ N(0, 0.02^2) with 0.5% N(0, 0.2^2) outliers, {tokens} probe tokens "
                         "with 1% channels x20; forward error of w4a8_linear against fp32 x W^T",
             **out,
-            "speed_note": "the E2M1 grid runs through the same kernels as the codebook here (same bytes, "
-                          "same speed); native block-scaled FP4 tensor cores (kind::mxf4nvf4, 9 PFLOP/s dense "
-                          "nominal vs 2.23 measured for fp16 here) would also need 4-bit activations"}
+            "speed_note": "lloyd_max_codebook and e2m1_grid run through the codebook layer's kernels (same "
+                          "bytes, same speed); nvfp4_w4a4_* run the native block-scaled FP4 layer "
+                          "(other_configs.nvfp4_native has its speed)"}
+
+
+def _timed_replay(replay, stream, steps):
+    import torch
+    replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def measure_nvfp4(B, torch, dev, rank, stream, peaks, steps=30, dec_steps=2000, copies=4):
+    """Native NVFP4 layer (4-bit weights AND activations, tcgen05.mma
+    kind::mxf4nvf4) on the codebook layer's shape K=5120, N=17408: the weight
+    conversion, the prefill step (quantise + GEMM) and the GEMM alone at
+    M=4096, and decode calls at M=1 and 16 (64-token tile, no split-K) on
+    `copies` weight copies cycled (each 50 MB, together more than L2)."""
+    n, k = N_PRE, K_PRE
+    g = torch.Generator(device=dev)
+    g.manual_seed(31 + rank)
+    w = torch.randn((n, k), generator=g, device=dev) * 0.02
+    conv_ms = _timed_replay(lambda: [B.nvfp4_quantize(w, rotate=True, per_tensor=True) for _ in range(3)],
+                            stream, 3)
+    wc, wsf, gw = B.nvfp4_quantize(w, rotate=True, per_tensor=True)
+    del w
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    wbytes = n * k // 2 + n * k // 16 + 4 * n
+    out = {"workload": f"K={k} N={n}; weights fp32 N(0, 0.02^2) -> NVFP4 (rotated, one fp32 scalar per tensor)",
+           "convert_ms": conv_ms}
+    for m in (4096, 1, 16):
+        x = torch.randn((m, k), generator=g, device=dev).to(torch.bfloat16)
+        wsp = B.nvfp4_linear_workspace(m, k, dev)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        sets = [(wc, wsf, gw)] if m > 64 else [(wc.clone(), wsf.clone(), gw.clone()) for _ in range(copies)]
+        reps = steps if m > 64 else dec_steps
+        step = lambda i: B.nvfp4_linear(x, *sets[i % len(sets)], workspace=wsp, out=y)
+        for i in range(3):
+            step(i)
+        lin_ms = _timed_replay(graph_loop(step, reps, stream), stream, reps)
+        xc, xs, gx = B.nvfp4_quantize(x, rotate=True)
+        gstep = lambda i: B.nvfp4_gemm(xc, xs, gx, *sets[i % len(sets)], out=y)
+        gemm_ms = _timed_replay(graph_loop(gstep, reps, stream), stream, reps)
+        flops = 2.0 * m * n * k
+        if m > 64:
+            tf = flops / (gemm_ms * 1e-3) / 1e12
+            out[f"prefill_M{m}"] = {
+                "ms_per_step": lin_ms, "TOPS": flops / (lin_ms * 1e-3) / 1e12,
+                "roofline": {"kernel": "nvfp4_gemm_kernel<256>", "bound": "tensor", "achieved": tf,
+                             "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
+                             "peak_note": "measured dense bf16 burst peak x 4 (the nominal dense fp4/bf16 "
+                                          "ratio, 9 / 2.25 PFLOP/s)",
+                             "ms_per_launch": gemm_ms}}
+        else:
+            gb = wbytes / (gemm_ms * 1e-3) / 1e9
+            out[f"decode_M{m}"] = {
+                "us_per_step": lin_ms * 1e3, "step_GBs": wbytes / (lin_ms * 1e-3) / 1e9,
+                "roofline": {"kernel": "nvfp4_gemm_kernel<64>", "bound": "hbm", "achieved": gb,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gb / peaks["hbm_gbs"],
+                             "us_per_launch": gemm_ms * 1e3,
+                             "bytes": "codes 0.5 B + scales 1/16 B per weight + 4 B per row"}}
+        del sets, x, wsp, y, xc, xs, gx
+    del wc, wsf, gw
+    torch.cuda.empty_cache()
+    return out
 
 
 def main() -> None:
@@ -721,6 +797,7 @@ def main() -> None:
     ap.add_argument("--prefill-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the C2/C3/second-prefill lines")
+    ap.add_argument("--only", default="", help="comma-separated subset of the other configurations to run")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="reference arm: about how long warm-up plus timed steps take in all")
     args = ap.parse_args()
@@ -943,13 +1020,20 @@ def main() -> None:
 
     # ---------------- the other configurations: C2 token sweep, C3 decode step, C4 second shape
     extra = {}
+    only = {s for s in args.only.split(",") if s}
+    runs = {
+        "c2_down_proj": lambda: measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup),
+        "c1_streaming_rate": lambda: measure_c1_rate(B, synth, torch, dev, rank, stream),
+        "c3_decode_step": lambda: measure_c3(B, synth, torch, dev, rank, stream, 20, 3),
+        "c4_prefill_8192": lambda: measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3),
+        "weight_converter": lambda: measure_converter(B, torch, dev, rank, stream),
+        "nvfp4_foil": lambda: measure_nvfp4_foil(B, torch, dev, rank),
+        "nvfp4_native": lambda: measure_nvfp4(B, torch, dev, rank, stream, peaks),
+    }
     if not args.no_extra:
-        extra["c2_down_proj"] = measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup)
-        extra["c1_streaming_rate"] = measure_c1_rate(B, synth, torch, dev, rank, stream)
-        extra["c3_decode_step"] = measure_c3(B, synth, torch, dev, rank, stream, 20, 3)
-        extra["c4_prefill_8192"] = measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3)
-        extra["weight_converter"] = measure_converter(B, torch, dev, rank, stream)
-        extra["nvfp4_foil"] = measure_nvfp4_foil(B, torch, dev, rank)
+        for name, run in runs.items():
+            if not only or name in only:
+                extra[name] = run()
     err = B.get_device_error()
 
     if world > 1:

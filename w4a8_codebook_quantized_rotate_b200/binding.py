@@ -511,6 +511,13 @@ def nvfp4_gemm(x_codes: torch.Tensor, x_scales: torch.Tensor, g_x: torch.Tensor,
     return out
 
 
+def nvfp4_linear_workspace(m: int, k: int, device) -> torch.Tensor:
+    nbytes = int(load_library().w4a8_nvfp4_linear_workspace_bytes(m, k))
+    if nbytes == 0:
+        raise W4A8Error("w4a8_nvfp4_linear_workspace_bytes", 2)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
 def nvfp4_linear(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, g_w: torch.Tensor,
                  workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
                  stream=None) -> torch.Tensor:

@@ -291,4 +291,45 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 
+// ---------------------------------------------------------------- transposed bf16 epilogue
+
+// One warp stores a 32 x 32 block of a row-major bf16 matrix y [M, N]: rows
+// (tokens) mc .. mc + 31, columns (outputs) nb .. nb + 31, where thread i
+// holds column nb + i for the 32 rows (value(j) is row mc + j, as bf16
+// bits).  The block goes through 2 KiB of shared memory [row][column], so
+// the global stores are 16 bytes of 8 consecutive columns (4 threads cover
+// the block's 64-byte run of a row) rather than one 2-byte store per value.
+// Rows >= M and columns >= N are not written.
+template <typename Value>
+__device__ __forceinline__ void store_block_transposed(uint16_t* __restrict__ y, int M, int N, int mc, int nb,
+                                                       uint32_t tbuf, int lane, Value value) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint16_t b = value(j);
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(tbuf + uint32_t(j) * 64u + uint32_t(lane) * 2u), "h"(b));
+  }
+  __syncwarp();
+  const bool vec = (N & 7) == 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = lane + 32 * i, row = idx >> 2, part = idx & 3;
+    const int m = mc + row, n = nb + 8 * part;
+    if (m < M && n < N) {
+      uint32_t w[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                   : "r"(tbuf + uint32_t(row) * 64u + uint32_t(part) * 16u));
+      uint16_t* dst = y + size_t(m) * N + n;
+      if (vec) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (n + e < N) dst[e] = uint16_t(w[e >> 1] >> (16 * (e & 1)));
+      }
+    }
+  }
+  __syncwarp();
+}
+
 }  // namespace w4a8

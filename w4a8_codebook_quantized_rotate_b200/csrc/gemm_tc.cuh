@@ -308,21 +308,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       pdl_wait();  // s_x comes from the previous kernel
       const float sch = valid ? p.sch[n] : 0.f;
+      // every stage is free once the accumulator is complete: stage 0 holds each warp's 32 x 32 bf16 block
+      const uint32_t tbuf = bstage0 + uint32_t(warp - 2) * 2048u;
 #pragma unroll 1
-      for (int ci = grp * (kTcTokens / 64); ci < (grp + 1) * (kTcTokens / 64); ++ci) {
+      for (int ci = grp * (kTcTokens / 64); ci < (grp + 1) * (kTcTokens / 64) && m0 + 32 * ci < p.M; ++ci) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + trow + kTcAccCol + uint32_t(ci) * 32u, v);
         tc_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int m = m0 + ci * 32 + j;
-            if (m < p.M) {
-              const float val = __uint_as_float(v[j]) * sch * p.s_x[m];
-              p.y[size_t(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-            }
-          }
-        }
+        const int mc = m0 + 32 * ci;
+        store_block_transposed(p.y, p.M, p.N, mc, n0 + 32 * q, tbuf, lane, [&](int j) {
+          const float sx = mc + j < p.M ? p.s_x[mc + j] : 0.f;
+          return __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * sch * sx));
+        });
       }
     }
   }

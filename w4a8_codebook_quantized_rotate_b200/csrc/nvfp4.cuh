@@ -191,7 +191,7 @@ __global__ void nvfp4_pack_scales_kernel(const uint8_t* __restrict__ rows, int R
 
 // ------------------------------------------------------------------ GEMM
 
-template <int NT>
+template <int NT, int CPS = 1>  // CPS: CTAs resident per SM (each takes its share of shared memory and TMEM)
 struct NvCfg {
   static constexpr uint32_t kA = kNvRows * 128;                 // weight codes: 128 rows x 128 bytes
   static constexpr uint32_t kB = NT * 128;                      // token codes
@@ -199,7 +199,9 @@ struct NvCfg {
   static constexpr int kSfbBlocks = (NT + 127) / 128;           // 128-row scale blocks of the token tile
   static constexpr uint32_t kSfb = kSfbBlocks * 4 * kNvSfChunk;
   static constexpr uint32_t kStage = kA + kB + kSfa + kSfb;     // a multiple of 1024
-  static constexpr int kStages = int((kNvMaxSmem - 2048) / kStage) > 8 ? 8 : int((kNvMaxSmem - 2048) / kStage);
+  // a CTA's share of the SM's 228 KiB (1 KiB of each CTA's share is reserved)
+  static constexpr size_t kBudget = CPS == 1 ? kNvMaxSmem : size_t(233472 / CPS) - 1024;
+  static constexpr int kStages = int((kBudget - 2048) / kStage) > 8 ? 8 : int((kBudget - 2048) / kStage);
   static constexpr size_t kSmem = 2048 + size_t(kStages) * kStage;
   static constexpr uint32_t kSfaCols = 16;                      // 4 steps x 4 columns
   static constexpr uint32_t kSfbStepCols = 4 * kSfbBlocks;      // columns of one k64 step's token scales
@@ -208,7 +210,11 @@ struct NvCfg {
   // K-major both, N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64.
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(NT >> 3) << 17) | (uint32_t(kNvRows >> 4) << 24);
   static_assert(kStage % 1024 == 0, "stages stay 1024-byte aligned");
-  static_assert(NT + kStages * kSfCols <= kNvTmemCols, "accumulator and scale columns fit the allocation");
+  // TMEM columns: the accumulator, then each stage's scale columns; a power of two of at least 32
+  static constexpr uint32_t kCols = NT + kStages * kSfCols;
+  static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
+  static_assert(kCols <= kNvTmemCols / CPS, "accumulator and scale columns fit the SM's share");
+  static_assert(kStages >= 2, "a pipeline");
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "token tile");
 };
 
@@ -275,11 +281,32 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// Epilogue of one warp: its 32 accumulator lanes (rows nb .. nb + 31) x NT
+// columns (tokens m0 ..), 32 columns at a time, stored through shared memory
+// (store_block_transposed).
 template <int NT>
-__global__ void __launch_bounds__(kNvThreads, 1)
+__device__ __forceinline__ void nv_epilogue(const NvGemmParams& p, uint32_t tmem_rows, uint32_t tbuf, int nb, int m0,
+                                            int lane) {
+  const int n = nb + lane;
+  const float gw = n < p.N ? p.gw[n] : 0.f;
+#pragma unroll 1
+  for (int c = 0; c < NT / 32 && m0 + 32 * c < p.M; ++c) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tmem_rows + uint32_t(32 * c), v);
+    tc_wait_ld();
+    const int mc = m0 + 32 * c;
+    store_block_transposed(p.y, p.M, p.N, mc, nb, tbuf, lane, [&](int j) {
+      const float gx = mc + j < p.M ? p.gx[mc + j] : 0.f;
+      return __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * gw * gx));
+    });
+  }
+}
+
+template <int NT, int CPS = 1>
+__global__ void __launch_bounds__(kNvThreads, CPS)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                       const NvGemmParams p) {
-  using C = NvCfg<NT>;
+  using C = NvCfg<NT, CPS>;
   extern __shared__ __align__(1024) uint8_t nv_smem[];
   pdl_launch_dependents();
   NvShared* sh = reinterpret_cast<NvShared*>(nv_smem);
@@ -300,7 +327,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sh->tmem_base, kNvTmemCols);
+    tmem_alloc(&sh->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -391,35 +418,19 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   } else {
     // ------------------------------------------------ epilogue: y[m, n] = D[n, m] g_w[n] g_x[m]
     const int q = warp & 3;  // the TMEM lane quarter this warp may read
-    const int n = n0 + 32 * q + lane;
-    const bool valid = n < p.N;
     const int acc_ok = lane == 0 ? int(nv_wait(&sh->acc_full, 0, sh, p.err)) : 0;
     if (__shfl_sync(0xffffffffu, acc_ok, 0) != 0) {
       tc_fence_after();
       pdl_wait();  // g_x comes from the previous kernel
-      const float gw = valid ? p.gw[n] : 0.f;
-#pragma unroll 1
-      for (int c = 0; c < NT / 32 && m0 + 32 * c < p.M; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(32 * c), v);
-        tc_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int m = m0 + 32 * c + j;
-            if (m < p.M) {
-              const float val = __uint_as_float(v[j]) * gw * p.gx[m];
-              p.y[size_t(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-            }
-          }
-        }
-      }
+      // every stage is free once the accumulator is complete: stage 0 holds each warp's 32 x 32 bf16 block
+      const uint32_t tbuf = stage0 + uint32_t(q) * 2048u;
+      nv_epilogue<NT>(p, tmem + (uint32_t(32 * q) << 16), tbuf, n0 + 32 * q, m0, lane);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kNvTmemCols);
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 }  // namespace w4a8

@@ -92,6 +92,7 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(nvfp4_quant_kernel, size_t(kMaxK) * 4) != cudaSuccess ||
           allow_smem(nvfp4_gemm_kernel<256>, NvCfg<256>::kSmem) != cudaSuccess ||
           allow_smem(nvfp4_gemm_kernel<128>, NvCfg<128>::kSmem) != cudaSuccess ||
+          allow_smem(nvfp4_gemm_kernel<128, 2>, NvCfg<128, 2>::kSmem) != cudaSuccess ||
           allow_smem(nvfp4_gemm_kernel<64>, NvCfg<64>::kSmem) != cudaSuccess)
         return W4A8_ERR_CUDA;
     }
@@ -950,6 +951,17 @@ w4a8_status w4a8_decode_chain(const w4a8_chain_layer* layers, int64_t n_layers, 
 
 // ------------------------------------------------------------------ NVFP4 comparison layer
 
+#ifndef W4A8_NV_PREFILL_NT
+#define W4A8_NV_PREFILL_NT 128
+#endif
+#ifndef W4A8_NV_PREFILL_CPS
+#define W4A8_NV_PREFILL_CPS 2
+#endif
+constexpr int kNvPrefillNT = W4A8_NV_PREFILL_NT;    // token tile beyond 128 tokens
+constexpr int kNvPrefillCPS = W4A8_NV_PREFILL_CPS;  // its CTAs per SM
+static_assert((kNvPrefillNT == 256 && kNvPrefillCPS == 1) || (kNvPrefillNT == 128 && kNvPrefillCPS <= 2),
+              "a compiled prefill configuration");
+
 static bool nv_shape_ok(int64_t R, int64_t K) {
   return R > 0 && R <= (int64_t(1) << 24) && K > 0 && K % kNvBK == 0 && K <= kMaxK;
 }
@@ -1008,7 +1020,9 @@ static w4a8_status nv_gemm(const uint8_t* x_codes, const uint8_t* x_scales, cons
                            uint16_t* y, const DeviceState* d, cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return W4A8_ERR_CUDA;
-  const int nt = M > 128 ? 256 : M > 64 ? 128 : 64;
+  // token tile: 64 / 128 for few tokens (one CTA per SM); beyond, the prefill tile
+  const int nt = M > 128 ? kNvPrefillNT : M > 64 ? 128 : 64;
+  const int cps = M > 128 ? kNvPrefillCPS : 1;
   CUtensorMap tw, tx;
   const cuuint64_t gw_dim[2] = {cuuint64_t(K / 2), cuuint64_t(N)};
   const cuuint64_t gx_dim[2] = {cuuint64_t(K / 2), cuuint64_t(M)};
@@ -1037,6 +1051,8 @@ static w4a8_status nv_gemm(const uint8_t* x_codes, const uint8_t* x_scales, cons
   cudaError_t e;
   if (nt == 256)
     e = launch_pdl(nvfp4_gemm_kernel<256>, grid, dim3(kNvThreads), NvCfg<256>::kSmem, s, tw, tx, p);
+  else if (nt == 128 && cps == 2)
+    e = launch_pdl(nvfp4_gemm_kernel<128, 2>, grid, dim3(kNvThreads), NvCfg<128, 2>::kSmem, s, tw, tx, p);
   else if (nt == 128)
     e = launch_pdl(nvfp4_gemm_kernel<128>, grid, dim3(kNvThreads), NvCfg<128>::kSmem, s, tw, tx, p);
   else
