@@ -769,16 +769,18 @@ def measure_nvfp4(B, torch, dev, rank, stream, peaks, steps=30, dec_steps=2000, 
             tf = flops / (gemm_ms * 1e-3) / 1e12
             out[f"prefill_M{m}"] = {
                 "ms_per_step": lin_ms, "TOPS": flops / (lin_ms * 1e-3) / 1e12,
-                "roofline": {"kernel": "nvfp4_gemm_kernel<256>", "bound": "tensor", "achieved": tf,
+                "roofline": {"kernel": "nvfp4_gemm_kernel<128, 2>", "bound": "tensor", "achieved": tf,
                              "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
                              "peak_note": "measured dense bf16 burst peak x 4 (the nominal dense fp4/bf16 "
                                           "ratio, 9 / 2.25 PFLOP/s)",
+                             "traffic": profiled_traffic("nvfp4_gemm_kernel_prefill",
+                                                         ["nvfp4.cuh", "act.cuh", "common.cuh"]),
                              "ms_per_launch": gemm_ms}}
         else:
             gb = wbytes / (gemm_ms * 1e-3) / 1e9
             out[f"decode_M{m}"] = {
                 "us_per_step": lin_ms * 1e3, "step_GBs": wbytes / (lin_ms * 1e-3) / 1e9,
-                "roofline": {"kernel": "nvfp4_gemm_kernel<64>", "bound": "hbm", "achieved": gb,
+                "roofline": {"kernel": "nvfp4_gemm_kernel<64, 1>", "bound": "hbm", "achieved": gb,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gb / peaks["hbm_gbs"],
                              "us_per_launch": gemm_ms * 1e3,
                              "bytes": "codes 0.5 B + scales 1/16 B per weight + 4 B per row"}}
@@ -1028,7 +1030,8 @@ def main() -> None:
         "c4_prefill_8192": lambda: measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3),
         "weight_converter": lambda: measure_converter(B, torch, dev, rank, stream),
         "nvfp4_foil": lambda: measure_nvfp4_foil(B, torch, dev, rank),
-        "nvfp4_native": lambda: measure_nvfp4(B, torch, dev, rank, stream, peaks),
+        "nvfp4_native": lambda: measure_nvfp4(B, torch, dev, rank, stream, peaks, steps=max(3, args.prefill_steps),
+                                              dec_steps=min(2000, args.steps)),
     }
     if not args.no_extra:
         for name, run in runs.items():

@@ -22,7 +22,8 @@ def test_committed_traffic_matches_its_source_hash():
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         d = json.load(f)
     files = {"decode_one_kernel_fused": ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"],
-             "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"]}
+             "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"],
+             "nvfp4_gemm_kernel_prefill": ["nvfp4.cuh", "act.cuh", "common.cuh"]}
     for kernel, srcs in files.items():
         if kernel not in d:
             assert bench.profiled_traffic(kernel, srcs) is None
@@ -30,8 +31,9 @@ def test_committed_traffic_matches_its_source_hash():
         got = bench.profiled_traffic(kernel, srcs)
         if d[kernel]["source_sha256_16"] == bench.kernel_source_hash(srcs):
             assert got == pytest.approx(d[kernel]["dram_bytes_per_launch"])
-            # both captures are of launches that read the whole 50.2 MB layer at least once
-            assert got >= bench.weight_bytes(17408, 5120)
+            # every capture is of a launch that reads a whole 17408 x 5120 layer (its 4-bit codes
+            # and e4m3 scales, 50.1 MB) at least once
+            assert got >= 17408 * 5120 * (0.5 + 1 / 16)
         else:
             assert got is None
 

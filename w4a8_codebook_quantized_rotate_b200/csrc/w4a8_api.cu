@@ -984,7 +984,8 @@ static w4a8_status nv_quantize(const void* x, int32_t x_is_f32, int64_t R, int64
   p.rotate = rotate ? 1 : 0;
   if (amax_word) {
     if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned), s) != cudaSuccess) return W4A8_ERR_CUDA;
-    nvfp4_amax_kernel<<<unsigned(R), kNvQuantThreads, 0, s>>>(p, amax_word);
+    const unsigned grid = unsigned(std::min<int64_t>(R, int64_t(d->sms) * 8));
+    nvfp4_amax_kernel<<<grid, kNvQuantThreads, 0, s>>>(p, amax_word);
     if (launch_status() != W4A8_OK) return W4A8_ERR_CUDA;
   }
   const unsigned rows = unsigned((R + 127) / 128 * 128);
