@@ -382,12 +382,14 @@ def c2_path(m: int, k: int, n: int) -> str:
     """Which kernel w4a8_linear runs for (M, K, N) (the library's rule)."""
     if m == 1:
         return "one-token decode (activation step fused)"
-    if 64 <= m <= 128 and (n + 127) // 128 < 100:
+    if 65 <= m <= 128 and (n + 127) // 128 < 100:
         return "small-batch tensor-core (stream-K)"
     if m <= 16:
         return "decode"
+    if m <= 32:
+        return "decode, 32-token variant"
     if m <= 64:
-        return "decode, slices of 16"
+        return "decode, slices of 32"
     return "tensor-core GEMM"
 
 

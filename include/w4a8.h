@@ -140,9 +140,10 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  *   packed     a buffer filled by w4a8_pack_layout for the same (N, K).
  *   y          output [M, N] bf16 bit patterns (uint16), row-major.
  *   workspace  scratch of at least w4a8_linear_workspace_bytes(M, K, N).
- * M <= 64 runs the decode kernel (a weight-streaming GEMV, one launch per
- * slice of up to 16 tokens); larger M runs the tensor-core GEMM, except that
- * 64 <= M <= 128 on a layer of fewer than 100 row tiles of 128 (where the
+ * M <= 64 runs the decode kernel (a weight-streaming GEMV: one launch for
+ * up to 16 tokens, else one per slice of up to 32); larger M runs the
+ * tensor-core GEMM, except that
+ * 65 <= M <= 128 on a layer of fewer than 100 row tiles of 128 (where the
  * GEMM would leave most SMs idle) runs a small-batch tensor-core kernel
  * that splits the weight stream over every SM.  For one token a single
  * kernel rotates, quantises and applies the layer (every CTA quantises the

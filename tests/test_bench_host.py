@@ -75,8 +75,11 @@ def test_oracle_pool_splits_rows_over_processes():
 def test_c2_path_names_follow_the_library_rule():
     assert bench.c2_path(1, 17408, 5120).startswith("one-token")
     assert bench.c2_path(4, 17408, 5120) == "decode"
-    assert bench.c2_path(32, 17408, 5120) == "decode, slices of 16"
-    assert bench.c2_path(64, 17408, 5120).startswith("small-batch")
+    assert bench.c2_path(16, 17408, 5120) == "decode"
+    assert bench.c2_path(17, 17408, 5120) == "decode, 32-token variant"
+    assert bench.c2_path(32, 17408, 5120) == "decode, 32-token variant"
+    assert bench.c2_path(64, 17408, 5120) == "decode, slices of 32"
+    assert bench.c2_path(65, 17408, 5120).startswith("small-batch")
     assert bench.c2_path(128, 17408, 5120).startswith("small-batch")
     assert bench.c2_path(128, 5120, 17408) == "tensor-core GEMM"
     assert bench.c2_path(256, 17408, 5120) == "tensor-core GEMM"

@@ -212,6 +212,10 @@ __global__ void __launch_bounds__(kActMaxThreads) rotate_quant_kernel(const uint
 // quant_code): the same codes and s_x.  Splitting the token over up to 8
 // SMs cuts the latency of the step before a decode GEMV.
 constexpr int kActClusterBlocks = 16;  // 256-blocks per CTA (one per warp)
+
+// Blocks of 8 tokens of a decode launch of m tokens: 1 (up to 8), 2 (up to
+// 16) or 4 (up to 32) -- the decode kernel's variants.
+__host__ __device__ constexpr int dec_blocks(int m) { return m <= 8 ? 1 : m <= 16 ? 2 : 4; }
 constexpr int kActClusterThreads = kActClusterBlocks * 32;
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -236,14 +240,16 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t ra
   return v;
 }
 
-// Tokens are laid out in slices of 16 (the decode kernel runs one launch per
-// slice): token m goes to slice m / 16, `slice_half2` half2 units apart, as
-// token m % 16 of a slice with ceil(tokens in the slice / 8) blocks of 8.
+// Tokens are laid out in slices of `slice_m` (16 or 32; the decode kernel
+// runs one launch per slice): token m goes to slice m / slice_m,
+// `slice_half2` half2 units apart, as token m % slice_m of a slice with
+// dec_blocks(tokens in the slice) blocks of 8 (1, 2 or 4: the decode
+// kernel's variants).
 // The first CTA also clears `zero_count` 16-byte words at `zero_vec` (the
 // decode workspace's split-K counters).
 __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_kernel(
     const uint16_t* __restrict__ x, int M, int K, __half2* __restrict__ out, float* __restrict__ s_x,
-    int slice_half2, uint4* __restrict__ zero_vec, int zero_count) {
+    int slice_half2, uint4* __restrict__ zero_vec, int zero_count, int slice_m) {
   __shared__ float warp_max[kActClusterBlocks];
   __shared__ float cta_max;
   // The previous kernel may still read the workspace: wait before writing.
@@ -280,9 +286,8 @@ __global__ void __launch_bounds__(kActClusterThreads) rotate_quant_frag_cluster_
   const QuantScale qs = quant_prepare(s);
   if (rank == 0 && threadIdx.x == 0) s_x[m] = s;
   if (mine) {
-    const int sl = m >> 4, ml = m & 15;
-    const int in_slice = min(16, M - 16 * sl);
-    const int nb = (in_slice + 7) >> 3;
+    const int sl = m / slice_m, ml = m - sl * slice_m;
+    const int nb = dec_blocks(min(slice_m, M - slice_m * sl));
     __half2* o = out + int64_t(sl) * slice_half2;
     const int k0 = b * kRotBlock + lane * 8;
     auto put = [&](auto fast) {

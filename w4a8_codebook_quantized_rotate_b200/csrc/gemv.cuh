@@ -21,6 +21,10 @@
 //     following odd chunk accumulate into one fragment whose columns are
 //     the 8 group partials of each row, and each lane scales its 4 of them
 //     by s_rel in fp32 once per chunk pair (instead of once per step);
+//   * 17..32 tokens (four blocks of 8 per fragment): the group scale goes
+//     into the fragment instead, fp16(fp16(cb) s_rel) as in the prefill
+//     kernel, and the MMAs accumulate in fp32 -- 4 multiplies per k16 step
+//     instead of 4 per token block;
 //   * s_x and s_ch scale the final sum in fp32, and y is rounded to bf16.
 //
 // Work split ("stream-K"): a unit is (tile pair p, chunk c), i.e. 32 rows x
@@ -47,7 +51,13 @@ namespace w4a8 {
 constexpr int kDecWarps = 16;                      // one token
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecWarpsMulti = 12;                 // 2..16 tokens: fewer warps, more registers each
+constexpr int kDecWarpsWide = 8;                   // 17..32 tokens (4 blocks of 8): more registers still
 __host__ __device__ constexpr int dec_warps(bool single) { return single ? kDecWarps : kDecWarpsMulti; }
+// Warps per CTA of the kernel serving m tokens (one launch).
+__host__ __device__ constexpr int dec_warps_m(int m) {
+  return m == 1 ? kDecWarps : m <= 16 ? kDecWarpsMulti : kDecWarpsWide;
+}
+__host__ __device__ constexpr int dec_warps_nb(int nb) { return nb >= 4 ? kDecWarpsWide : kDecWarpsMulti; }
 constexpr int kDecTG = 2;                          // tiles (16 rows each) per unit
 constexpr int kDecMaxCtas = 148;                   // cap on the grid, fixes the workspace size
 // The part of a workspace that must hold zeros when a launch starts (every
@@ -63,6 +73,7 @@ constexpr int kDecSchRows = 1024;                  // row scales staged in share
 // Units in flight per warp (register ring depth) per variant.
 constexpr int kDecDepth1 = 3;                      // 2..8 tokens
 constexpr int kDecDepth2 = 2;                      // 9..16 tokens
+constexpr int kDecDepth4 = 3;                      // 17..32 tokens
 
 struct DecodeParams {
   const uint16_t* x;     // one token's bf16 activations [K] (the kernel that rotates and quantises them itself)
@@ -110,8 +121,9 @@ __host__ __device__ inline int dec_slot_floats(int m) { return kDecTG * 16 * m; 
 // Dynamic shared memory of a launch: table (+ alignment room), one token's
 // activations, and the CTA's per-warp partials.
 __host__ __device__ inline size_t dec_smem_bytes(int m, int k, bool single) {
-  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(dec_warps(single)) * 2 * dec_slot_floats(m) * 4 +
-         kDecSchRows * 4 + 64 + 128 + 64;
+  return kDecSmemBase + (single ? size_t(k) * 2 : 0) + size_t(single ? kDecWarps : dec_warps_m(m)) * 2 *
+         dec_slot_floats(m) * 4 +
+         kDecSchRows * 4 + 128 + 128 + 64;
 }
 
 
@@ -252,15 +264,35 @@ __device__ __forceinline__ void dec_compute(const DecStage<NB>& st, float (&acc)
 #pragma unroll
       for (int i = 0; i < kDecTG; ++i) {
         const uint32_t pair_codes = ((s < 2) ? st.s[i].x : st.s[i].y) >> (16 * (s & 1));
-        const float2 sc = e4m3x2_to_float2(pair_codes);  // (row g, row g+8)
+        if constexpr (NB >= 4) {
+          // Four token blocks share each fragment: scale the fragment once
+          // (fp16(fp16(cb) s_rel), the prefill kernel's operand) and let the
+          // MMAs accumulate in fp32, instead of rescaling 4 NB partials.
+          __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(pair_codes & 0xFFFFu), __NV_E4M3);
+          const __half2 hh = *reinterpret_cast<const __half2*>(&hr);  // (row g, row g+8), exact
+          const __half2 sg = __low2half2(hh), sg8 = __high2half2(hh);
+          uint32_t as[4];
+          const __half2 m0 = __hmul2(*reinterpret_cast<const __half2*>(&a[i][s2][0]), sg);
+          const __half2 m1 = __hmul2(*reinterpret_cast<const __half2*>(&a[i][s2][1]), sg8);
+          const __half2 m2 = __hmul2(*reinterpret_cast<const __half2*>(&a[i][s2][2]), sg);
+          const __half2 m3 = __hmul2(*reinterpret_cast<const __half2*>(&a[i][s2][3]), sg8);
+          as[0] = *reinterpret_cast<const uint32_t*>(&m0);
+          as[1] = *reinterpret_cast<const uint32_t*>(&m1);
+          as[2] = *reinterpret_cast<const uint32_t*>(&m2);
+          as[3] = *reinterpret_cast<const uint32_t*>(&m3);
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          float d[4];
-          mma_16816z(d, a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b[s2][j][0], b[s2][j][1], zero);
-          acc[i][j][0] = fmaf(d[0], sc.x, acc[i][j][0]);
-          acc[i][j][2] = fmaf(d[2], sc.y, acc[i][j][2]);
-          acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
-          acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
+          for (int j = 0; j < NB; ++j) mma_16816(acc[i][j], as[0], as[1], as[2], as[3], b[s2][j][0], b[s2][j][1]);
+        } else {
+          const float2 sc = e4m3x2_to_float2(pair_codes);  // (row g, row g+8)
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            float d[4];
+            mma_16816z(d, a[i][s2][0], a[i][s2][1], a[i][s2][2], a[i][s2][3], b[s2][j][0], b[s2][j][1], zero);
+            acc[i][j][0] = fmaf(d[0], sc.x, acc[i][j][0]);
+            acc[i][j][2] = fmaf(d[2], sc.y, acc[i][j][2]);
+            acc[i][j][1] = fmaf(d[1], sc.x, acc[i][j][1]);
+            acc[i][j][3] = fmaf(d[3], sc.y, acc[i][j][3]);
+          }
         }
       }
     }
@@ -381,7 +413,7 @@ struct DecWaitPdl {
 
 template <int NB, int D, class Wait>
 __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& wait_inputs) {
-  constexpr int kW = dec_warps(false);
+  constexpr int kW = dec_warps_nb(NB);
   constexpr int kThr = kW * 32;
   extern __shared__ __align__(16) uint8_t dec_smem[];
   const uint32_t base = smem_u32(dec_smem);
@@ -389,8 +421,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
   const uint32_t parts = lut + 65536u;                // [warp][2] partials
   const uint32_t part_bytes = uint32_t(dec_slot_floats(p.M)) * 4u;
   const uint32_t sch_s = parts + uint32_t(kW * 2) * part_bytes;  // row scales
-  const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..16)
-  const uint32_t wbeg_s = sx_s + 64;  // warp range starts [17]; at +96 the CTA pair context [4]
+  const uint32_t sx_s = sch_s + kDecSchRows * 4;                          // s_x[0..32)
+  const uint32_t wbeg_s = sx_s + 128;  // warp range starts [kW + 1]; at +96 the CTA pair context [4]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int cta_w0 = blockIdx.x * kW;
   const int w = cta_w0 + wl;
@@ -625,7 +657,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
 }
 
 template <int NB, int D>
-__global__ void __launch_bounds__(dec_warps(false) * 32, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(dec_warps_nb(NB) * 32, 1) decode_kernel(const DecodeParams p) {
   // The next kernel may launch now: it streams its own weights and waits for
   // this grid's completion before it touches anything this grid writes.
   pdl_launch_dependents();

@@ -87,6 +87,7 @@ w4a8_status device_state(DeviceState** out) {
           allow_smem(decode_chain_kernel, dec_smem_bytes(1, kMaxK, true)) != cudaSuccess ||
           allow_smem(decode_kernel<1, kDecDepth1>, dec_smem_bytes(8, kMaxK, false)) != cudaSuccess ||
           allow_smem(decode_kernel<2, kDecDepth2>, dec_smem_bytes(16, kMaxK, false)) != cudaSuccess ||
+          allow_smem(decode_kernel<4, kDecDepth4>, dec_smem_bytes(32, kMaxK, false)) != cudaSuccess ||
           allow_smem(gemm_tc_kernel, kTcSmemBytes) != cudaSuccess ||
           allow_smem(gemm_sk_kernel, 232448) != cudaSuccess ||  // the largest sk_smem_bytes over token tiles
           allow_smem(nvfp4_quant_kernel, size_t(kMaxK) * 4) != cudaSuccess ||
@@ -107,15 +108,19 @@ w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK
 
 // ------------------------------------------------------------------ linear workspace
 
-// One token runs the one-token decode kernel, 2..64 tokens the mma.sync
-// decode kernel in slices of up to 16 tokens, more the prefill GEMM -- except
-// that 64..128 tokens on a layer with few 128-row tiles (the GEMM would leave
-// most SMs idle: 40 CTAs at N = 5120) run the small-batch tensor-core kernel,
-// which splits the weight stream over every SM.
-constexpr int kDecodeSliceM = 16;
+// One token runs the one-token decode kernel, 2..16 tokens the mma.sync
+// decode kernel in one launch, 17..64 in launches of up to 32 tokens, more
+// the prefill GEMM -- except that 65..128 tokens on a layer with few 128-row
+// tiles (the GEMM would leave most SMs idle: 40 CTAs at N = 5120) run the
+// small-batch tensor-core kernel, which splits the weight stream over every
+// SM.  (Measured at K = 17408, N = 5120: 32 tokens 42 us in one launch
+// against 52 us in two of 16; 64 tokens 76 us in two launches of 32 against
+// 99 us on the small-batch kernel.)
+constexpr int kDecodeSliceM = 16;      // the slice of up to 16 tokens (also the static-scratch limit)
+constexpr int kDecodeWideSliceM = 32;  // the slice when M > 16
 constexpr int kDecodeMaxM = 64;
 #ifndef W4A8_SK_MIN_M
-#define W4A8_SK_MIN_M 64
+#define W4A8_SK_MIN_M 65
 #endif
 constexpr int64_t kSkMinM = W4A8_SK_MIN_M;
 constexpr int64_t kSkMaxRowTiles = 100;  // more 128-row tiles than this keep the GEMM busy enough
@@ -129,7 +134,8 @@ struct LinearPlan {
   int nt;          // sk: token tile (M rounded up to 16)
   size_t off_part; // sk: partial tiles
   int nb;          // decode: token blocks of 8 of a full slice
-  int slices;      // decode: launches of up to kDecodeSliceM tokens
+  int slice_m;     // decode: tokens per launch (16 up to 16 tokens, else 32)
+  int slices;      // decode: launches of up to slice_m tokens
   size_t slice_bytes;  // decode: B-fragment bytes of one slice
   size_t off_sx, off_xq, off_slots, total;  // [0, kWsZeroBytes): exchange words and counters
   int T, P, C;
@@ -143,9 +149,10 @@ LinearPlan linear_plan(int64_t M, int64_t K, int64_t N, bool allow_sk = true) {
   L.C = int(K / kChunkK);
   L.P = (L.T + kDecTG - 1) / kDecTG;
   if (L.decode) {
-    const int64_t mslice = M < kDecodeSliceM ? M : kDecodeSliceM;
-    L.nb = int((mslice + 7) / 8);
-    L.slices = int((M + kDecodeSliceM - 1) / kDecodeSliceM);
+    L.slice_m = M <= kDecodeSliceM ? kDecodeSliceM : kDecodeWideSliceM;
+    const int64_t mslice = M < L.slice_m ? M : L.slice_m;
+    L.nb = dec_blocks(int(mslice));
+    L.slices = int((M + L.slice_m - 1) / L.slice_m);
     L.slice_bytes = size_t(K) * L.nb * 16;
     L.off_sx = kWsZeroBytes;
     L.off_xq = L.off_sx + 256;  // s_x: at most 64 floats
@@ -352,8 +359,8 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
                                  unsigned* x_ready = nullptr) {
   const PackedLayout L = packed_layout(N, K);
   for (int sl = 0; sl < plan.slices; ++sl) {
-    const int64_t m0 = int64_t(sl) * kDecodeSliceM;
-    const int64_t ms = M - m0 < kDecodeSliceM ? M - m0 : kDecodeSliceM;
+    const int64_t m0 = int64_t(sl) * plan.slice_m;
+    const int64_t ms = M - m0 < plan.slice_m ? M - m0 : plan.slice_m;
     DecodeParams p{};  // the decode-chain fields stay null
     p.x = x;
     p.units = pk + L.off_units;
@@ -374,7 +381,7 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     p.T = plan.T;
     p.P = plan.P;
     p.U = plan.P * plan.C;
-    const int wpc = dec_warps(ms == 1);  // warps per CTA of this variant
+    const int wpc = dec_warps_m(int(ms));  // warps per CTA of this variant
     const int ctas_avail = d->sms < kDecMaxCtas ? d->sms : kDecMaxCtas;
     const int warps_avail = ctas_avail * wpc;
     p.W = p.U < warps_avail ? p.U : warps_avail;
@@ -383,7 +390,7 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
     one_token_split(p, ctas_avail);
     const dim3 grid(ms == 1 ? unsigned(p.G) : unsigned((p.W + wpc - 1) / wpc));
     const size_t smem = dec_smem_bytes(int(ms), int(K), ms == 1);
-    const int nb = int((ms + 7) / 8);
+    const int nb = dec_blocks(int(ms));
     cudaError_t e;
     if (x && K > kDecPairK)  // pairs of CTAs share the activation step (an even grid; extra CTAs hold no units)
       e = launch_pdl_cluster(decode_one_kernel<true>, dim3((grid.x + 1) & ~1u), dim3(kOneThreads), 2, smem, s, p);
@@ -393,8 +400,10 @@ static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, i
       e = launch_pdl(decode_one_kernel<false>, grid, dim3(kOneThreads), smem, s, p);
     else if (nb == 1)
       e = launch_pdl(decode_kernel<1, kDecDepth1>, grid, dim3(wpc * 32), smem, s, p);
-    else
+    else if (nb == 2)
       e = launch_pdl(decode_kernel<2, kDecDepth2>, grid, dim3(wpc * 32), smem, s, p);
+    else
+      e = launch_pdl(decode_kernel<4, kDecDepth4>, grid, dim3(wpc * 32), smem, s, p);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
   }
   return W4A8_OK;
@@ -419,7 +428,7 @@ static w4a8_status prepare_impl(const uint16_t* x, int64_t M, int64_t K, int64_t
     if (launch_pdl_cluster(rotate_quant_frag_cluster_kernel, dim3(cl, unsigned(M)), dim3(kActClusterThreads), cl, 0,
                            s, x, int(M), int(K), reinterpret_cast<__half2*>(ws + plan.off_xq), s_x,
                            int(plan.slice_bytes / 4), reinterpret_cast<uint4*>(ws + zero_from),
-                           int((kWsZeroBytes - zero_from) / 16)) != cudaSuccess)
+                           int((kWsZeroBytes - zero_from) / 16), plan.slice_m) != cudaSuccess)
       return W4A8_ERR_CUDA;
   } else {
     if (launch_pdl(rotate_quant_kernel<kActF16Row>, dim3(unsigned(M)), dim3(act_threads(K)), size_t(K) * 4, s, x,
