@@ -339,13 +339,40 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       old = __shfl_sync(0xffffffffu, old, 0);
       if (old != unsigned(last - first)) return true;  // another CTA finishes this share
       __threadfence();
-      for (int m = col0; m < col0 + half && m < p.M; ++m) {
-        float tot = 0.f;
-        for (int cc = first; cc <= last; ++cc) {
-          const int sl = cc * 2 + (sk_cta_item(cc, p) >= seg_tile * p.C ? 0 : 1);
-          tot += __ldcg(p.part + (size_t(sl) * p.NT + m) * kSkRows + r);
+      // Sum the CTAs' partials in CTA order.  Loads go out 8 tokens x 4 CTAs
+      // at a time (a token-by-token loop waits one L2 round trip per token:
+      // measured 28-50 us of a 105-129 us call).
+      const int m_end = min(col0 + half, p.M);
+      for (int mc = col0; mc < m_end; mc += 8) {
+        float tot[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) tot[jj] = 0.f;
+        for (int c0 = first; c0 <= last; c0 += 4) {
+          float v[4][8];
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int cc = c0 + qq;
+            const bool have = cc <= last;
+            const int sl = have ? cc * 2 + (sk_cta_item(cc, p) >= seg_tile * p.C ? 0 : 1) : 0;
+            const float* src = p.part + (size_t(sl) * p.NT + mc) * kSkRows + r;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) v[qq][jj] = (have && mc + jj < m_end) ? __ldcg(src + jj * kSkRows) : 0.f;
+          }
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq)
+            if (c0 + qq <= last) {  // only the CTAs that exist: the same additions as one at a time
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) tot[jj] += v[qq][jj];
+            }
         }
-        if (valid) p.y[size_t(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(tot * sch * p.s_x[m]));
+        if (valid) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int m = mc + jj;
+            if (m < m_end)
+              p.y[size_t(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(tot[jj] * sch * p.s_x[m]));
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) *cnt = 0u;  // ready for the next launch on this workspace
