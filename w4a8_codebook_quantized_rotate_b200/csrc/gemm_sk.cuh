@@ -74,11 +74,14 @@ struct SkParams {
   uint32_t idesc;
 };
 
+// One barrier pair per stage (an x_q tile in shared memory and a weight slot
+// in TMEM): `full` counts the TMA thread's transfer and the 128 expansion
+// threads of the group that filled the slot, `empty` is the MMA thread's
+// commit.  The MMA thread waits once and commits once per item (two waits
+// and two commits per item cost the prefill kernel ~10 %).
 struct SkShared {
-  uint64_t b_full[kSkMaxStagesB];
-  uint64_t b_empty[kSkMaxStagesB];
-  uint64_t a_full[kSkStagesA];
-  uint64_t a_empty[kSkStagesA];
+  uint64_t full[kSkStagesA];
+  uint64_t empty[kSkStagesA];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
@@ -143,16 +146,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int i1 = sk_cta_item(min(int(blockIdx.x) + 1, p.G), p);
   const int n_items = i1 - i0;
   const bool dbl = p.NT <= 128;  // two accumulators fit beside the A stages
-  const int SB = sk_stages_b(p.NT);
+  // stages: as many x_q tiles as fit in shared memory, at most the 8 TMEM weight slots
+  const int SB = sk_stages_b(p.NT) < kSkStagesA ? sk_stages_b(p.NT) : kSkStagesA;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SB; ++s) {
-      mbar_init(&sh->b_full[s], 1);
-      mbar_init(&sh->b_empty[s], 1);
-    }
-    for (int s = 0; s < kSkStagesA; ++s) {
-      mbar_init(&sh->a_full[s], 128);
-      mbar_init(&sh->a_empty[s], 1);
+      mbar_init(&sh->full[s], 129);  // the TMA thread + 128 expansion threads
+      mbar_init(&sh->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->acc_full[b], 1);
@@ -206,16 +206,22 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       int kb = i0 % p.C, issued = 0;
       for (int j = 0; j < n_items; ++j) {
         const int s = j % SB;
-        if (!sk_wait(&sh->b_empty[s], ((j / SB) & 1) ^ 1, sh, p.err)) break;
-        mbar_arrive_expect_tx(&sh->b_full[s], stage_b);
-        tma_load_2d(bstage0 + uint32_t(s) * stage_b, &tmap_x, &sh->b_full[s], kb * kTcBK, 0);
+        if (!sk_wait(&sh->empty[s], ((j / SB) & 1) ^ 1, sh, p.err)) break;
+        mbar_arrive_expect_tx(&sh->full[s], stage_b);
+        tma_load_2d(bstage0 + uint32_t(s) * stage_b, &tmap_x, &sh->full[s], kb * kTcBK, 0);
         ++issued;
         if (++kb == p.C) kb = 0;
         if (j + kSkPfItems < n_items) prefetch_item(i0 + j + kSkPfItems);
       }
-      if (sh->abort) {  // let copies already in flight land before the CTA exits
-        for (int i = issued > SB ? issued - SB : 0; i < issued; ++i)
-          mbar_wait_bounded(&sh->b_full[i % SB], (i / SB) & 1, p.err, 1u << 20);
+      if (sh->abort && issued > 0) {
+        // The stage barriers also count the expansion threads, which may have
+        // stopped: let the copies in flight land by waiting a fixed, bounded
+        // time (a tile lands in microseconds) before the CTA exits.
+        unsigned long long t0, t1;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        do {
+          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+        } while (t1 - t0 < 50000ull);  // 50 us
       }
     }
   } else if (warp == 1) {
@@ -224,26 +230,24 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       bool ok = true;
       int kb = i0 % p.C, seg = 0;
       for (int j = 0; j < n_items && ok; ++j) {
-        const int sa = j % kSkStagesA, sb = j % SB;
+        const int sa = j % SB;
         const int buf = dbl ? (seg & 1) : 0;
         const int use = dbl ? (seg >> 1) : seg;  // earlier segments on this buffer
         if (j == 0 || kb == 0) {  // a segment starts: its accumulator must be drained
           ok = use == 0 || sk_wait(&sh->acc_empty[buf], (use - 1) & 1, sh, p.err);
           if (!ok) break;
         }
-        ok = sk_wait(&sh->a_full[sa], (j / kSkStagesA) & 1, sh, p.err) &&
-             sk_wait(&sh->b_full[sb], (j / SB) & 1, sh, p.err);
+        ok = sk_wait(&sh->full[sa], (j / SB) & 1, sh, p.err);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(buf) * uint32_t(p.NT);
 #pragma unroll
         for (int s = 0; s < kTcBK / 16; ++s) {
           const uint32_t a = tmem + kSkACol + uint32_t(sa) * 32u + uint32_t(s) * 8u;
-          const uint64_t bd = sw128_desc(bstage0 + uint32_t(sb) * stage_b + uint32_t(s) * 32u);
+          const uint64_t bd = sw128_desc(bstage0 + uint32_t(sa) * stage_b + uint32_t(s) * 32u);
           tc_mma_ts_f16(acc, a, bd, p.idesc, ((j == 0 || kb == 0) && s == 0) ? 0u : 1u);
         }
-        tc_commit(&sh->a_empty[sa]);
-        tc_commit(&sh->b_empty[sb]);
+        tc_commit(&sh->empty[sa]);
         if (++kb == p.C || j == n_items - 1) {  // the segment ends
           tc_commit(&sh->acc_full[buf]);
           kb = kb == p.C ? 0 : kb;
@@ -394,7 +398,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         return false;
       }
       if (!ok) return false;
-      const int sa = jj % kSkStagesA;
+      const int sa = jj % SB;
       uint32_t v[32];
       const int n = row_of(jt);
       exp_compute(es[i], lut_lane, (n >> 3) & 1, v);
@@ -408,14 +412,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const int nn = row_of(t);
         sk_exp_load(es[i], p, nn >> 4, k, nn & 7, jj + 2 * PF < n_items && nn < p.N);
       }
-      int w_ok = lane == 0 ? int(sk_wait(&sh->a_empty[sa], ((jj / kSkStagesA) & 1) ^ 1, sh, p.err)) : 0;
+      int w_ok = lane == 0 ? int(sk_wait(&sh->empty[sa], ((jj / SB) & 1) ^ 1, sh, p.err)) : 0;
       ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
       if (!ok) return false;
       tc_fence_after();
       tmem_st_32x32b_x32(tmem + trow + kSkACol + uint32_t(sa) * 32u, v);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&sh->a_full[sa]);
+      mbar_arrive(&sh->full[sa]);
       jk += 2;
       if (jk >= p.C) { jk -= p.C; ++jt; }
       return true;
