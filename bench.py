@@ -382,7 +382,7 @@ def c2_path(m: int, k: int, n: int) -> str:
     """Which kernel w4a8_linear runs for (M, K, N) (the library's rule)."""
     if m == 1:
         return "one-token decode (activation step fused)"
-    if 65 <= m <= 128 and (n + 127) // 128 < 100:
+    if 65 <= m <= 256 and (n + 127) // 128 < 100:
         return "small-batch tensor-core (stream-K)"
     if m <= 16:
         return "decode"
@@ -395,8 +395,9 @@ def c2_path(m: int, k: int, n: int) -> str:
 
 def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
     """Down-projection shape K=17408, N=5120 at several token counts, 8 weight
-    copies cycled: M <= 64 runs the decode kernel (one launch per 16 tokens),
-    larger M the GEMM; the per-call time shows where the GEMM takes over."""
+    copies cycled; `path` names the kernel each count takes (c2_path); the
+    per-call and per-token times show the crossover from the weight-bound
+    decode kernels to the tensor-core kernels."""
     k, n = 17408, 5120
     copies = []
     for c in range(COPIES):
@@ -405,7 +406,7 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
         del q
     wbytes = weight_bytes(n, k)
     out = {}
-    for m in (1, 4, 16, 32, 64, 128):
+    for m in (1, 4, 16, 32, 64, 128, 256):
         g = torch.Generator(device=dev)
         g.manual_seed(300 + m)
         x = torch.randn((m, k), generator=g, device=dev).to(torch.bfloat16)

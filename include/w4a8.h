@@ -143,7 +143,7 @@ size_t w4a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  * M <= 64 runs the decode kernel (a weight-streaming GEMV: one launch for
  * up to 16 tokens, else one per slice of up to 32); larger M runs the
  * tensor-core GEMM, except that
- * 65 <= M <= 128 on a layer of fewer than 100 row tiles of 128 (where the
+ * 65 <= M <= 256 on a layer of fewer than 100 row tiles of 128 (where the
  * GEMM would leave most SMs idle) runs a small-batch tensor-core kernel
  * that splits the weight stream over every SM.  For one token a single
  * kernel rotates, quantises and applies the layer (every CTA quantises the

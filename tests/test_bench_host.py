@@ -82,4 +82,5 @@ def test_c2_path_names_follow_the_library_rule():
     assert bench.c2_path(65, 17408, 5120).startswith("small-batch")
     assert bench.c2_path(128, 17408, 5120).startswith("small-batch")
     assert bench.c2_path(128, 5120, 17408) == "tensor-core GEMM"
-    assert bench.c2_path(256, 17408, 5120) == "tensor-core GEMM"
+    assert bench.c2_path(256, 17408, 5120).startswith("small-batch")
+    assert bench.c2_path(257, 17408, 5120) == "tensor-core GEMM"

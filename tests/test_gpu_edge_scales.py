@@ -13,7 +13,8 @@ kernel's cluster-pair path):
     7.5.
 Each runs through the one-token kernel (activation step fused, and the
 two-kernel path), the 2..16-token kernel, the sliced path (17..64 tokens),
-the small-batch tensor-core kernel (64..128 tokens on a narrow layer) and
+the small-batch tensor-core kernel (65..256 tokens on a narrow layer; 256
+tokens take its single-accumulator path) and
 the tensor-core GEMM, against the oracle at the layer's bars.
 """
 
@@ -65,7 +66,8 @@ def _check(y, y_ref, x, wmax):
 @pytest.mark.parametrize("kind", ["converted", "stored"])
 @pytest.mark.parametrize("k", [5120, 17408])
 @pytest.mark.parametrize("m,path", [(1, "fused"), (1, "two_kernel"), (4, "decode"), (16, "decode"),
-                                    (40, "sliced"), (100, "small_batch"), (300, "gemm")])
+                                    (40, "sliced"), (100, "small_batch"), (256, "small_batch_single_acc"),
+                                    (300, "gemm")])
 def test_edge_layers_every_path(lib, kind, k, m, path):
     q, packed, wmax = _layer(lib, kind, k)
     bits, x, _ = synth.activations(m, k, synth.rng_for(42, m, "act"), k // 100)

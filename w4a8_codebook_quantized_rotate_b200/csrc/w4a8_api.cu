@@ -110,12 +110,13 @@ w4a8_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A8_OK
 
 // One token runs the one-token decode kernel, 2..16 tokens the mma.sync
 // decode kernel in one launch, 17..64 in launches of up to 32 tokens, more
-// the prefill GEMM -- except that 65..128 tokens on a layer with few 128-row
+// the prefill GEMM -- except that 65..256 tokens on a layer with few 128-row
 // tiles (the GEMM would leave most SMs idle: 40 CTAs at N = 5120) run the
 // small-batch tensor-core kernel, which splits the weight stream over every
 // SM.  (Measured at K = 17408, N = 5120: 32 tokens 42 us in one launch
 // against 52 us in two of 16; 64 tokens 76 us in two launches of 32 against
-// 99 us on the small-batch kernel.)
+// 99 us on the small-batch kernel; 256 tokens 108 us on the small-batch kernel
+// against 128 us on the GEMM.)
 constexpr int kDecodeSliceM = 16;      // the slice of up to 16 tokens (also the static-scratch limit)
 constexpr int kDecodeWideSliceM = 32;  // the slice when M > 16
 constexpr int kDecodeMaxM = 64;
@@ -124,7 +125,7 @@ constexpr int kDecodeMaxM = 64;
 #endif
 constexpr int64_t kSkMinM = W4A8_SK_MIN_M;
 constexpr int64_t kSkMaxRowTiles = 100;  // more 128-row tiles than this keep the GEMM busy enough
-constexpr int64_t kSkMaxM = 128;         // measured: ahead of the GEMM at 64 and 128 tokens, behind at 256
+constexpr int64_t kSkMaxM = 256;         // its largest token tile (measured ahead of the GEMM up to there)
 
 static_assert(size_t(kSkMaxCtas) * 8 * 4 <= kWsXchBytes, "the small-batch counters fit in the zero region");
 
