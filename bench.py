@@ -429,8 +429,11 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / st
         out[f"M={m}"] = {"us_per_call": us, "weight_GBs": wbytes / us / 1e3,
-                         "us_per_token": us / m,
+                         "us_per_token": us / m, "TOPS": 2.0 * m * n * k / us / 1e6,
                          "path": c2_path(m, k, n)}
+        if m == 128:  # the small-batch kernel's DRAM bytes from its committed capture at this size
+            out[f"M={m}"]["traffic"] = profiled_traffic("gemm_sk_kernel_m128",
+                                                        ["gemm_sk.cuh", "gemm_tc.cuh", "common.cuh"])
         del replay
     del copies
     torch.cuda.empty_cache()
@@ -1027,7 +1030,7 @@ def main() -> None:
     extra = {}
     only = {s for s in args.only.split(",") if s}
     runs = {
-        "c2_down_proj": lambda: measure_c2(B, synth, torch, dev, rank, stream, 2000, args.warmup),
+        "c2_down_proj": lambda: measure_c2(B, synth, torch, dev, rank, stream, min(2000, args.steps), args.warmup),
         "c1_streaming_rate": lambda: measure_c1_rate(B, synth, torch, dev, rank, stream),
         "c3_decode_step": lambda: measure_c3(B, synth, torch, dev, rank, stream, 20, 3),
         "c4_prefill_8192": lambda: measure_c4b(B, synth, torch, dev, rank, stream, max(3, args.prefill_steps // 2), 3),

@@ -23,7 +23,8 @@ def test_committed_traffic_matches_its_source_hash():
         d = json.load(f)
     files = {"decode_one_kernel_fused": ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"],
              "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"],
-             "nvfp4_gemm_kernel_prefill": ["nvfp4.cuh", "act.cuh", "common.cuh"]}
+             "nvfp4_gemm_kernel_prefill": ["nvfp4.cuh", "act.cuh", "common.cuh"],
+             "gemm_sk_kernel_m128": ["gemm_sk.cuh", "gemm_tc.cuh", "common.cuh"]}
     for kernel, srcs in files.items():
         if kernel not in d:
             assert bench.profiled_traffic(kernel, srcs) is None
