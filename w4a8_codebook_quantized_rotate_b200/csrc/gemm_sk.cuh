@@ -1,4 +1,5 @@
-// Small-batch kernel (2 <= M <= 256 tokens): the tensor-core GEMM of
+// Small-batch kernel (65..256 tokens on a layer of few 128-row tiles; it
+// accepts 2..256): the tensor-core GEMM of
 // gemm_tc.cuh with one token tile sized to M and a stream-K split of the
 // weight stream over every SM.
 //

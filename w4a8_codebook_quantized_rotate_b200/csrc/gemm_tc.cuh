@@ -1,4 +1,5 @@
-// Prefill kernel (M > 16): tensor-core GEMM on tcgen05 with the codebook
+// Prefill kernel (M > 64; on a layer of few 128-row tiles, M > 256):
+// tensor-core GEMM on tcgen05 with the codebook
 // expansion fused into the operand path.
 //
 // The product is computed transposed, D^T[n, m] = sum_k W'[n, k] x_q[m, k],

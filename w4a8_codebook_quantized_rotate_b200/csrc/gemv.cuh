@@ -1,4 +1,4 @@
-// Decode kernel (M <= 16): y[m, n] = s_x[m] s_ch[n] sum_g s_rel[n, g] sum_{k in g} cb[idx[n, k]] x_q[m, k].
+// Decode kernel (2 <= M <= 32 per launch): y[m, n] = s_x[m] s_ch[n] sum_g s_rel[n, g] sum_{k in g} cb[idx[n, k]] x_q[m, k].
 //
 // The layer re-reads every weight for every token, so this kernel is bound
 // by HBM ("Qwen3.8-27B-AEON-ULTIMATE-UNCENSORED-BF16 -- W4A8 ConvRot for
@@ -15,12 +15,8 @@
 //     and up to 8 tokens; a k16 step is exactly one 16-wide group, so its
 //     fp32 partial is scaled by the group's s_rel in fp32 and accumulated in
 //     fp32;
-//   * for one token the MMA's 8 columns hold 8 groups instead of 8 tokens:
-//     in k16 step s of chunk c only the lanes of column 4 (c & 1) + s carry
-//     x (the B operand is zero elsewhere), so the steps of an even and the
-//     following odd chunk accumulate into one fragment whose columns are
-//     the 8 group partials of each row, and each lane scales its 4 of them
-//     by s_rel in fp32 once per chunk pair (instead of once per step);
+//   * (one token runs gemv1.cuh, whose MMA columns hold 8 groups instead of
+//     8 tokens, so each lane scales its group partials once per chunk pair);
 //   * 17..32 tokens (four blocks of 8 per fragment): the group scale goes
 //     into the fragment instead, fp16(fp16(cb) s_rel) as in the prefill
 //     kernel, and the MMAs accumulate in fp32 -- 4 multiplies per k16 step
@@ -29,16 +25,14 @@
 //
 // Work split ("stream-K"): a unit is (tile pair p, chunk c), i.e. 32 rows x
 // 64 k.  The P * C units, in [p][c] order (the order they lie in memory),
-// are cut into W equal ranges, one per warp; a CTA's 16 warps hold 16
-// consecutive ranges.  A warp that covers a whole tile pair writes y
-// directly.  A pair split between warps is reduced in two levels, both in a
-// fixed order (the result is deterministic): the warps of a CTA leave their
-// partials in shared memory and one warp adds them after a CTA barrier.  A
-// pair that also crosses into one other CTA (one token) is joined through
-// one 64-bit exchange word per row, and the second CTA to arrive adds the
-// two sums (two fp32 terms: the same in either order); otherwise each CTA
-// leaves its partial in the workspace and the last to finish (an atomic
-// counter, no waiting) adds them in CTA order and writes y.
+// are cut into W equal ranges, one per warp; a CTA's 12 (8 for 17..32
+// tokens) warps hold consecutive ranges.  A warp that covers a whole tile
+// pair writes y directly.  A pair split between warps is reduced in two
+// levels, both in a fixed order (the result is deterministic): the warps of
+// a CTA leave their partials in shared memory and one warp adds them after a
+// CTA barrier; a pair that also crosses into other CTAs leaves each CTA's
+// partial in the workspace, and the last CTA to finish (an atomic counter,
+// no waiting) adds them in CTA order and writes y.
 #pragma once
 
 #include <type_traits>
@@ -404,7 +398,7 @@ __device__ __forceinline__ void dec_zero(float (&acc)[kDecTG][NB][4]) {
 // partials in shared memory and one warp adds them after a CTA barrier; a
 // pair that also crosses into other CTAs is finished by the CTA that comes
 // last to it (an arrival counter; the last CTA adds the partials in CTA
-// order).  This kernel serves 2..16 tokens per launch; one token runs the
+// order).  This kernel serves 2..32 tokens per launch; one token runs the
 // kernel in gemv1.cuh.
 struct DecWaitPdl {
   static constexpr int kLoadsAhead = 4;  // kept blocks whose loads are all issued before the first transform

@@ -352,7 +352,8 @@ static void one_token_split(DecodeParams& p, int ctas_avail) {
   p.Dr = duos % p.G;
 }
 
-// Decode launch (M <= 16).  With x given (one token) the kernel also rotates
+// Decode launches (M <= 64, one per slice of plan.slice_m tokens).  With x
+// given (one token) the kernel also rotates
 // and quantises the token; otherwise it reads what w4a8_linear_prepare left
 // in the workspace.
 static w4a8_status launch_decode(const LinearPlan& plan, const DeviceState* d, int64_t M, int64_t K, int64_t N,
