@@ -27,8 +27,9 @@
  *     failed check nothing is launched and the status says why.
  *   - Shapes: K must be a multiple of 256 (the rotation block; a layer whose
  *     input width is not, such as 4304 = 16 x 269, stays unquantised on the
- *     pages) and at most W4A8_MAX_K; N must be a positive multiple of 16;
- *     M must be positive.
+ *     pages) and at most W4A8_MAX_K; N must be a positive multiple of 16,
+ *     at most 2^24; M must be positive and at most 16 776 960 (65535 tiles of
+ *     256 tokens).
  *   - Every pointer must be 16-byte aligned.
  *   - The calls run on the current CUDA device, which must be sm_100.
  */
@@ -398,7 +399,8 @@ w4a8_status w4a8_dense_reference(const uint16_t* x, int64_t M, int64_t K, const 
  *           of (row r, 16-block c) is byte 16 (r % 32) + 4 ((r % 128) / 32)
  *           + c % 4.  Pad rows hold 0.
  *   g       fp32 [R].
- * Shapes: R, M, N in [1, 2^24]; K a multiple of 256, at most W4A8_MAX_K.
+ * Shapes: R, N in [1, 2^24]; M in [1, 8 388 480] (65535 tiles of 128
+ * tokens); K a multiple of 256, at most W4A8_MAX_K.
  * Pointers 16-byte aligned.  Calls are asynchronous on `stream`.
  * ------------------------------------------------------------------------ */
 

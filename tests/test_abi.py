@@ -87,6 +87,8 @@ def test_nvfp4_refuses_bad_arguments_before_any_launch(lib):
     assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 256, 1, 1, fake, fake, fake, None, None) == 1
     assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 100, 1, 0, fake, fake, fake, None, None) == 2
     assert lib.w4a8_nvfp4_linear(fake, 4, 256, fake, fake, fake, 128, fake, fake, 16, None) == 4
+    # the GEMM's grid holds at most 65535 token tiles of 128
+    assert lib.w4a8_nvfp4_gemm(fake, fake, fake, 65535 * 128 + 1, fake, fake, fake, 128, 256, fake, None) == 2
 
 
 # Every workspace starts with the words that join partial sums across CTAs:
@@ -96,6 +98,9 @@ ZERO_REGION_BYTES = (148 * 32 * 8 + 148 * 4 + 255) // 256 * 256
 
 def test_workspace_sizes(lib):
     assert lib.w4a8_linear_workspace_bytes(0, 256, 16) == 0
+    # token counts stop at 65535 GEMM tiles of 256
+    assert lib.w4a8_linear_workspace_bytes(65535 * 256, 256, 16) > 0
+    assert lib.w4a8_linear_workspace_bytes(65535 * 256 + 1, 256, 16) == 0
     dec = lib.w4a8_linear_workspace_bytes(1, 5120, 17408)
     pre = lib.w4a8_linear_workspace_bytes(4096, 5120, 17408)
     assert dec > 5120 * 16 and pre >= 4096 * 5120 * 2 + 4096 * 4

@@ -52,8 +52,11 @@ bool weight_shape_ok(int64_t N, int64_t K) {
   return N > 0 && N % kTileRows == 0 && N <= (int64_t(1) << 24) && K > 0 && K % kRotBlock == 0 && K <= kMaxK;
 }
 
+// Token counts up to 65535 tiles of 256 (the GEMM's grid has one y index per token tile).
+constexpr int64_t kMaxTokens = int64_t(65535) * 256;
+
 bool act_shape_ok(int64_t M, int64_t K) {
-  return M > 0 && M <= (int64_t(1) << 24) && K > 0 && K % kRotBlock == 0 && K <= kMaxK;
+  return M > 0 && M <= kMaxTokens && K > 0 && K % kRotBlock == 0 && K <= kMaxK;
 }
 
 template <typename Kern>
@@ -1072,11 +1075,14 @@ static w4a8_status nv_gemm(const uint8_t* x_codes, const uint8_t* x_scales, cons
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
+// The GEMM's grid has one y index per token tile (up to 128 tokens each): at most 65535.
+constexpr int64_t kNvMaxTokens = int64_t(65535) * 128;
+
 w4a8_status w4a8_nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* g_x, int64_t M,
                             const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, int64_t N, int64_t K,
                             uint16_t* y, void* stream) {
   if (!x_codes || !x_scales || !g_x || !w_codes || !w_scales || !g_w || !y) return W4A8_ERR_NULL;
-  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K) || M > kNvMaxTokens) return W4A8_ERR_SHAPE;
   if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
     return W4A8_ERR_ALIGN;
   DeviceState* d = nullptr;
@@ -1104,7 +1110,7 @@ w4a8_status w4a8_nvfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uin
                               const uint8_t* w_scales, const float* g_w, int64_t N, uint16_t* y, void* workspace,
                               size_t workspace_bytes, void* stream) {
   if (!x || !w_codes || !w_scales || !g_w || !y || !workspace) return W4A8_ERR_NULL;
-  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K)) return W4A8_ERR_SHAPE;
+  if (!nv_shape_ok(M, K) || !nv_shape_ok(N, K) || M > kNvMaxTokens) return W4A8_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace))
     return W4A8_ERR_ALIGN;
   const NvLinearWs w = nv_linear_ws(M, K);
