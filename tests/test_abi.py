@@ -86,6 +86,7 @@ def test_nvfp4_refuses_bad_arguments_before_any_launch(lib):
     assert lib.w4a8_nvfp4_gemm(vp(4097), fake, fake, 16, fake, fake, fake, 128, 256, fake, None) == 3
     assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 256, 1, 1, fake, fake, fake, None, None) == 1
     assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 100, 1, 0, fake, fake, fake, None, None) == 2
+    assert lib.w4a8_nvfp4_quantize(fake, 0, 4, 256, 1, 1, fake, fake, fake, vp(4098), None) == 3
     assert lib.w4a8_nvfp4_linear(fake, 4, 256, fake, fake, fake, 128, fake, fake, 16, None) == 4
     # the GEMM's grid holds at most 65535 token tiles of 128
     assert lib.w4a8_nvfp4_gemm(fake, fake, fake, 65535 * 128 + 1, fake, fake, fake, 128, 256, fake, None) == 2

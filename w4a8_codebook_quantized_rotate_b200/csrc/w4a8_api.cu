@@ -1012,7 +1012,9 @@ w4a8_status w4a8_nvfp4_quantize(const void* x, int32_t x_is_f32, int64_t R, int6
                                 unsigned* amax_scratch, void* stream) {
   if (!x || !codes || !scales || !g || (per_tensor && !amax_scratch)) return W4A8_ERR_NULL;
   if (!nv_shape_ok(R, K)) return W4A8_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(g)) return W4A8_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(g) ||
+      (per_tensor && !aligned16(amax_scratch)))
+    return W4A8_ERR_ALIGN;
   return nv_quantize(x, x_is_f32, R, K, rotate, per_tensor ? amax_scratch : nullptr, codes, scales, g,
                      static_cast<cudaStream_t>(stream));
 }
