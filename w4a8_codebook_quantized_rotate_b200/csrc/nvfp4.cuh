@@ -18,18 +18,21 @@
 //   scales  the tensor core's order, rows padded to 128: chunks of 128 rows x
 //           64 k (512 bytes) in [row block][k64 step] order; inside a chunk
 //           the scale of (row r, 16-block c) is byte 16 (r % 32) +
-//           4 ((r % 128) / 32) + c % 4.  One tcgen05.cp 32x128b.warpx4 moves a
-//           chunk into four TMEM columns (row r -> lane r % 32 of every lane
-//           quarter, column (r % 128) / 32, byte c % 4), the layout the
-//           block-scaled MMA reads for M = 128 and scale_vec::4X.
+//           4 ((r % 128) / 32) + c % 4.  A chunk's 16-byte row i is the
+//           content of TMEM lane i (of every lane quarter) over four columns
+//           (row r -> lane r % 32, column (r % 128) / 32, byte c % 4), the
+//           layout the block-scaled MMA reads for M = 128 and scale_vec::4X.
 //   g       [R] fp32.
 //
 // GEMM: D^T[n, m] = sum_k W[n, k] x[m, k] with the weights as the MMA's A
 // operand (M = 128 rows, the TMEM lanes) and NT tokens as B; a stage is
 // 256 k: 128 bytes of codes per row by TMA (128-byte swizzle, no multicast),
 // the scale chunks by plain bulk copies, moved into per-stage TMEM columns by
-// the MMA thread before its four K = 64 MMAs.  The epilogue scales by
-// g_w[n] g_x[m] and stores bf16.
+// the four epilogue warps (tcgen05.st, each warp its lane quarter; with
+// tcgen05.cp issued by the MMA thread, 8 copies per stage held the tensor pipe
+// near a third busy), so the MMA thread waits once and issues its four
+// K = 64 MMAs per stage.  The epilogue scales by g_w[n] g_x[m] and stores
+// bf16.
 #pragma once
 
 #include <cuda.h>
@@ -238,7 +241,12 @@ struct NvGemmParams {
   int M, N, K;
 };
 
+// Per stage: `loaded` completes when the stage's code tiles and scale chunks
+// have landed (the TMA thread's transfer); `full` when the four epilogue
+// warps have moved the scale chunks into the stage's TMEM columns; `empty`
+// when the MMAs that read the stage have completed.
 struct NvShared {
+  uint64_t loaded[8];
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t acc_full;
@@ -266,16 +274,11 @@ __device__ __forceinline__ uint64_t nv_sw128_desc(uint32_t smem_addr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// Source descriptor of a 512-byte scale chunk for tcgen05.cp: no swizzle,
-// 8-row core matrices of 16-byte rows, 128 bytes apart; one core matrix wide.
-__device__ __forceinline__ uint64_t nv_sf_desc(uint32_t smem_addr) {
-  return uint64_t((smem_addr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 32) | (uint64_t(1) << 46);
-}
-
-// 32 rows x 16 bytes of shared memory -> 4 TMEM columns of lanes 0..31,
-// repeated in the other three lane quarters.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+// 32 lanes x 4 columns of 32-bit cells (thread i: lane quarter base + i).
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // D[tmem] (+)= (A * SFA) (B * SFB)^T, E2M1 operands from shared memory,
@@ -328,7 +331,8 @@ __global__ void __launch_bounds__(kNvThreads, CPS)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->loaded[s], 1);
+      mbar_init(&sh->full[s], 4);  // one arrival per epilogue warp
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->acc_full, 1);
@@ -363,13 +367,13 @@ __global__ void __launch_bounds__(kNvThreads, CPS)
       for (int kt = 0; kt < KT; ++kt) {
         if (!nv_wait(&sh->empty[s], phase ^ 1u, sh, p.err)) break;
         const uint32_t a = stage0 + uint32_t(s) * C::kStage;
-        mbar_arrive_expect_tx(&sh->full[s], bytes);
-        tma_load_2d(a, &tmap_w, &sh->full[s], kt * 128, n0);
-        tma_load_2d(a + C::kA, &tmap_x, &sh->full[s], kt * 128, m0);
-        bulk_load(a + C::kA + C::kB, sfa + size_t(kt) * 4 * kNvSfChunk, C::kSfa, &sh->full[s]);
+        mbar_arrive_expect_tx(&sh->loaded[s], bytes);
+        tma_load_2d(a, &tmap_w, &sh->loaded[s], kt * 128, n0);
+        tma_load_2d(a + C::kA, &tmap_x, &sh->loaded[s], kt * 128, m0);
+        bulk_load(a + C::kA + C::kB, sfa + size_t(kt) * 4 * kNvSfChunk, C::kSfa, &sh->loaded[s]);
         for (int i = 0; i < nb; ++i)
           bulk_load(a + C::kA + C::kB + C::kSfa + uint32_t(i) * 4u * kNvSfChunk,
-                    sfb + (size_t(i) * steps + size_t(kt) * 4) * kNvSfChunk, 4u * kNvSfChunk, &sh->full[s]);
+                    sfb + (size_t(i) * steps + size_t(kt) * 4) * kNvSfChunk, 4u * kNvSfChunk, &sh->loaded[s]);
         ++issued;
         if (++s == C::kStages) {
           s = 0;
@@ -398,15 +402,6 @@ __global__ void __launch_bounds__(kNvThreads, CPS)
         const uint32_t a = stage0 + uint32_t(s) * C::kStage;
         const uint32_t sfa_t = tmem + uint32_t(NT) + uint32_t(s) * C::kSfCols;
         const uint32_t sfb_t = sfa_t + C::kSfaCols;
-        const uint32_t sfa_s = a + C::kA + C::kB, sfb_s = sfa_s + C::kSfa;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tc_cp_32x128b_warpx4(sfa_t + 4u * j, nv_sf_desc(sfa_s + uint32_t(j) * kNvSfChunk));
-#pragma unroll
-          for (int i = 0; i < C::kSfbBlocks; ++i)
-            tc_cp_32x128b_warpx4(sfb_t + C::kSfbStepCols * j + 4u * i,
-                                 nv_sf_desc(sfb_s + uint32_t(i) * 4u * kNvSfChunk + uint32_t(j) * kNvSfChunk));
-        }
         const uint64_t ad = nv_sw128_desc(a), bd = nv_sw128_desc(a + C::kA);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -426,9 +421,52 @@ __global__ void __launch_bounds__(kNvThreads, CPS)
       }
     }
   } else {
-    // ------------------------------------------------ epilogue: y[m, n] = D[n, m] g_w[n] g_x[m]
-    const int q = warp & 3;  // the TMEM lane quarter this warp may read
-    const int acc_ok = lane == 0 ? int(nv_wait(&sh->acc_full, 0, sh, p.err)) : 0;
+    // ------------------------------------------------ scale chunks into TMEM, then the epilogue
+    const int q = warp & 3;  // the TMEM lane quarter this warp may access
+    // Per stage: every chunk (32 rows of 16 bytes: 128 rows x 4 scales of a k64 step) goes to 4 TMEM
+    // columns of this warp's 32 lanes; the four warps write the same data, which is the layout the
+    // block-scaled MMA reads (row r at lane r % 32 of every quarter, column (r % 128) / 32).  Moving
+    // them here keeps the MMA thread to one wait, four MMAs and one commit per stage.
+    bool ok = true;
+    {
+      int s = 0;
+      uint32_t phase = 0;
+      const uint32_t lanebase = uint32_t(32 * q) << 16;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const int w_ok = lane == 0 ? int(nv_wait(&sh->loaded[s], phase, sh, p.err)) : 0;
+        ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+        if (!ok) break;
+        const uint32_t sfa_s = stage0 + uint32_t(s) * C::kStage + C::kA + C::kB, sfb_s = sfa_s + C::kSfa;
+        const uint32_t sfa_t = tmem + lanebase + uint32_t(NT) + uint32_t(s) * C::kSfCols;
+        const uint32_t sfb_t = sfa_t + C::kSfaCols;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(sfa_s + uint32_t(j) * kNvSfChunk + uint32_t(lane) * 16u));
+          tmem_st_32x32b_x4(sfa_t + 4u * j, v);
+#pragma unroll
+          for (int i = 0; i < C::kSfbBlocks; ++i) {
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sfb_s + uint32_t(i) * 4u * kNvSfChunk + uint32_t(j) * kNvSfChunk +
+                               uint32_t(lane) * 16u));
+            tmem_st_32x32b_x4(sfb_t + C::kSfbStepCols * j + 4u * i, v);
+          }
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->full[s]);
+        if (++s == C::kStages) {
+          s = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // ---- epilogue: y[m, n] = D[n, m] g_w[n] g_x[m]
+    const int acc_ok = (ok && lane == 0) ? int(nv_wait(&sh->acc_full, 0, sh, p.err)) : 0;
     if (__shfl_sync(0xffffffffu, acc_ok, 0) != 0) {
       tc_fence_after();
       pdl_wait();  // g_x comes from the previous kernel
