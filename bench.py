@@ -912,15 +912,15 @@ def main() -> None:
     torch.cuda.synchronize()
     barrier()
     # (a) pipelined: step i's copy in, layer and copy out run on three streams
-    # with three buffer sets, so the copies of the neighbouring steps overlap
+    # with four buffer sets, so the copies of the neighbouring steps overlap
     # step i's layer; every step still moves its x in from pinned host memory
     # and its y out to pinned host memory.  The layer stream holds kernels
     # only (w4a8_linear_flagged waits on the GPU for a ready word the copy
     # writes after x), so consecutive layers keep their programmatic launch
     # overlap: a stream dependency on the copy event costs that overlap
     # (18.5 against 14.2 us per step, measured).  Captured in CUDA graphs of
-    # 128 steps (no overlap across graph boundaries).
-    NBUF = 3
+    # 512 steps (no overlap across graph boundaries).
+    NBUF = 4
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     xs = [torch.empty_like(x) for _ in range(NBUF)]
     ys = [torch.empty_like(y) for _ in range(NBUF)]
@@ -955,7 +955,7 @@ def main() -> None:
             side.wait_stream(s_out)
         return g
 
-    chunk = 128
+    chunk = 512
     pipe_graphs = [capture_pipelined(min(chunk, e2e_steps - b0), b0) for b0 in range(0, e2e_steps, chunk)]
     stream.wait_stream(side)
     torch.cuda.synchronize()
@@ -1104,7 +1104,7 @@ def main() -> None:
                 "how": "per step: pinned x copied in (then a ready word), w4a8_linear_flagged through the "
                        "Python binding (the layer waits on the GPU for the ready word, so its stream holds "
                        "kernels only), y copied out to pinned memory; copies on their own streams overlap the "
-                       "neighbouring steps' layers (three buffer sets); replayed from CUDA graphs of 128 steps",
+                       "neighbouring steps' layers (four buffer sets); replayed from CUDA graphs of 512 steps",
                 "host_loop": {"value": wbytes / (e2e_loop_ms * 1e-3) / 1e9 * world, "ms_per_step": e2e_loop_ms,
                               "how": "the same steps issued one by one from Python"}},
         "clocks": dec_clocks,
