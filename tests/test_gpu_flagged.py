@@ -76,3 +76,37 @@ def test_flagged_wait_runs_out_and_reports_a_timeout(lib):
     torch.cuda.synchronize()
     assert torch.equal(y.view(torch.int16), lib.linear(x, packed, n).view(torch.int16))
     assert lib.get_device_error() == 0
+
+
+def test_flagged_pipeline_of_distinct_tokens(lib):
+    """Consecutive one-token calls on one stream (so each may start while the
+    previous one runs), each token delivered by a copy and its ready word on
+    another stream into one of three buffer sets that are reused once the
+    call that read them is done.  Every step's output equals the plain
+    layer's on that token."""
+    m, k, n, steps, nbuf = 1, 5120, 4096, 12, 3
+    packed = _layer(lib, n, k, 11)
+    xs_host = [torch.randn((m, k)).mul(1 + i).to(torch.bfloat16).pin_memory() for i in range(steps)]
+    refs = [lib.linear(xh.cuda(), packed, n) for xh in xs_host]
+    one = torch.tensor([1, 0], dtype=torch.int32).pin_memory()
+    xs = [torch.zeros((m, k), dtype=torch.bfloat16, device="cuda") for _ in range(nbuf)]
+    flags = [torch.zeros(2, dtype=torch.int32, device="cuda") for _ in range(nbuf)]
+    ys = [torch.empty((m, n), dtype=torch.bfloat16, device="cuda") for _ in range(steps)]
+    done = [torch.cuda.Event() for _ in range(nbuf)]
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    comp, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        b = i % nbuf
+        if i >= nbuf:
+            copy.wait_event(done[b])  # the call that read this set is done
+        with torch.cuda.stream(copy):
+            xs[b].copy_(xs_host[i], non_blocking=True)
+            flags[b][:1].copy_(one[:1], non_blocking=True)
+        lib.linear_flagged(xs[b], packed, n, flags[b], ws, ys[i], stream=comp)
+        done[b].record(comp)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        assert torch.equal(ys[i].view(torch.int16), refs[i].view(torch.int16)), i
+    assert all(f.tolist() == [0, 0] for f in flags)
+    assert lib.get_device_error() == 0
