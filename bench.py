@@ -915,8 +915,8 @@ def main() -> None:
     # with four buffer sets, so the copies of the neighbouring steps overlap
     # step i's layer; every step still moves its x in from pinned host memory
     # and its y out to pinned host memory.  The layer stream holds kernels
-    # only (w4a8_linear_flagged waits on the GPU for a ready word the copy
-    # writes after x), so consecutive layers keep their programmatic launch
+    # only (w4a8_linear_flagged waits on the GPU for a ready word that the
+    # copy stream writes after x), so consecutive layers keep their programmatic launch
     # overlap: a stream dependency on the copy event costs that overlap
     # (18.5 against 14.2 us per step, measured).  Captured in CUDA graphs of
     # 512 steps (no overlap across graph boundaries).
@@ -926,7 +926,6 @@ def main() -> None:
     ys = [torch.empty_like(y) for _ in range(NBUF)]
     yh = [torch.empty((M_DEC, N_DEC), dtype=torch.bfloat16, pin_memory=True) for _ in range(NBUF)]
     flags = [torch.zeros(2, dtype=torch.int32, device=dev) for _ in range(NBUF)]
-    one_host = torch.tensor([1, 0], dtype=torch.int32).pin_memory()
     ev_comp = [torch.cuda.Event() for _ in range(NBUF)]
     ev_out = [torch.cuda.Event() for _ in range(NBUF)]
     side = torch.cuda.Stream()
@@ -944,7 +943,7 @@ def main() -> None:
                     s_in.wait_stream(side)
                 with torch.cuda.stream(s_in):
                     xs[b].copy_(x_host, non_blocking=True)
-                    flags[b][:1].copy_(one_host[:1], non_blocking=True)  # after x, same stream
+                B.signal_ready(flags[b], stream=s_in)  # the ready word, written by the stream after x
                 B.linear_flagged(xs[b], copies[(base + i) % COPIES], N_DEC, flags[b], ws, ys[b], stream=side)
                 ev_comp[b].record(side)
                 s_out.wait_event(ev_comp[b])
@@ -1101,7 +1100,8 @@ def main() -> None:
         "e2e": {"value": wbytes / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
                 "h2d_bytes_per_step": M_DEC * K_DEC * 2, "d2h_bytes_per_step": M_DEC * N_DEC * 2,
                 "ms_per_step": e2e_ms,
-                "how": "per step: pinned x copied in (then a ready word), w4a8_linear_flagged through the "
+                "how": "per step: pinned x copied in (then the ready word, written by the copy stream "
+                       "itself: w4a8_signal_ready), w4a8_linear_flagged through the "
                        "Python binding (the layer waits on the GPU for the ready word, so its stream holds "
                        "kernels only), y copied out to pinned memory; copies on their own streams overlap the "
                        "neighbouring steps' layers (four buffer sets); replayed from CUDA graphs of 512 steps",

@@ -186,6 +186,21 @@ w4a8_status w4a8_linear_flagged(const uint16_t* x, int64_t M, int64_t K,
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * Writes 1 to x_ready[0] in stream order: after everything issued earlier on
+ * `stream` (in particular the copy that brings x), with the ordering of a
+ * stream write of the driver (cuStreamWriteValue32, default flags: earlier
+ * writes of the stream are visible first).  The companion of
+ * w4a8_linear_flagged for a caller whose copy stream should carry x alone:
+ * the word is written by the stream itself, not copied from host memory.
+ * Can be captured into a CUDA graph.
+ *   x_ready  device, 2 words, 8-byte aligned (as for w4a8_linear_flagged);
+ *            only word 0 is written.
+ * Errors: W4A8_ERR_NULL, W4A8_ERR_ALIGN before anything is issued;
+ * W4A8_ERR_CUDA if the driver lacks the call or refuses it.
+ */
+w4a8_status w4a8_signal_ready(unsigned* x_ready, void* stream);
+
+/*
  * The two halves of w4a8_linear, for callers that apply several layers of
  * the same shape to one activation or that time the GEMM on its own.
  *

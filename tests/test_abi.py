@@ -36,8 +36,8 @@ def test_header_declares_the_boundary():
         "w4a8_linear_workspace_bytes", "w4a8_nvfp4_gemm", "w4a8_nvfp4_linear",
         "w4a8_nvfp4_linear_workspace_bytes", "w4a8_nvfp4_pack_scales", "w4a8_nvfp4_quantize",
         "w4a8_nvfp4_scale_bytes", "w4a8_pack_layout",
-        "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_selftest_timeout", "w4a8_status_string",
-        "w4a8_unpack_dequant"])
+        "w4a8_packed_bytes", "w4a8_rotate_quant_act", "w4a8_selftest_timeout", "w4a8_signal_ready",
+        "w4a8_status_string", "w4a8_unpack_dequant"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -134,6 +134,13 @@ def test_null_and_shape_errors_before_launch(lib):
     assert lib.w4a8_linear_run(1, 512, p, 16, None, p, 1 << 30, None) == 1
     assert lib.w4a8_linear_decode_static(None, 1, 256, p, 16, p, None) == 1
     assert lib.w4a8_linear_decode_static(p, 17, 256, p, 16, p, None) == 2
+
+
+def test_signal_ready_refuses_before_issuing(lib):
+    """A null or misaligned ready word is refused before the driver is asked
+    for anything (so this runs without a GPU)."""
+    assert lib.w4a8_signal_ready(None, None) == 1     # W4A8_ERR_NULL
+    assert lib.w4a8_signal_ready(4, None) == 3        # W4A8_ERR_ALIGN: not 8-byte aligned
 
 
 def test_status_strings(lib):

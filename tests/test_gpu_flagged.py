@@ -110,3 +110,58 @@ def test_flagged_pipeline_of_distinct_tokens(lib):
         assert torch.equal(ys[i].view(torch.int16), refs[i].view(torch.int16)), i
     assert all(f.tolist() == [0, 0] for f in flags)
     assert lib.get_device_error() == 0
+
+
+def test_ready_word_written_by_the_copy_stream(lib):
+    """w4a8_signal_ready after the copy of x on the copy stream: the layer,
+    launched first on its own stream, sees x complete."""
+    m, k, n = 1, 5120, 2048
+    packed = _layer(lib, n, k, 13)
+    x_host = torch.randn((m, k)).to(torch.bfloat16).pin_memory()
+    ref = lib.linear(x_host.cuda(), packed, n)
+    x_dev = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
+    ready = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    comp, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    lib.linear_flagged(x_dev, packed, n, ready, ws, y, stream=comp)
+    with torch.cuda.stream(copy):
+        x_dev.copy_(x_host, non_blocking=True)
+    lib.signal_ready(ready, stream=copy)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    assert ready.tolist() == [0, 0]
+    assert lib.get_device_error() == 0
+
+
+def test_ready_word_signal_in_a_captured_graph(lib):
+    """The copy, the stream-written ready word and the layer captured into one
+    CUDA graph (copy and layer on separate captured streams, no edge between
+    them), replayed with new tokens."""
+    m, k, n = 1, 5120, 2048
+    packed = _layer(lib, n, k, 14)
+    x_host = torch.empty((m, k), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
+    ready = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = lib.linear_workspace(m, k, n, "cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    side, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        copy.wait_stream(side)
+        with torch.cuda.stream(copy):
+            x_dev.copy_(x_host, non_blocking=True)
+        lib.signal_ready(ready, stream=copy)
+        lib.linear_flagged(x_dev, packed, n, ready, ws, y, stream=side)
+        side.wait_stream(copy)
+    torch.cuda.current_stream().wait_stream(side)
+    for rep in range(3):
+        x_host.copy_(torch.randn((m, k)).mul(rep + 1).to(torch.bfloat16))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = lib.linear(x_host.cuda(), packed, n)
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), rep
+        assert ready.tolist() == [0, 0]
+    assert lib.get_device_error() == 0

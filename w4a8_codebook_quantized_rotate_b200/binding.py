@@ -28,7 +28,7 @@ EXPORTS = (
     "w4a8_convert_workspace_bytes", "w4a8_convert_weight",
     "w4a8_compare_workspace_bytes", "w4a8_compare", "w4a8_dense_reference",
     "w4a8_chain_plan_bytes", "w4a8_chain_workspace_bytes", "w4a8_chain_plan", "w4a8_chain_run",
-    "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain", "w4a8_linear_flagged",
+    "w4a8_decode_chain_workspace_bytes", "w4a8_decode_chain", "w4a8_linear_flagged", "w4a8_signal_ready",
     "w4a8_nvfp4_scale_bytes", "w4a8_nvfp4_quantize", "w4a8_nvfp4_pack_scales", "w4a8_nvfp4_gemm",
     "w4a8_nvfp4_linear_workspace_bytes", "w4a8_nvfp4_linear",
 )
@@ -83,6 +83,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_decode_chain_workspace_bytes": (sz, [vp, i64]),
         "w4a8_decode_chain": (st, [vp, i64, vp, sz, vp]),
         "w4a8_linear_flagged": (st, [vp, i64, i64, vp, i64, vp, vp, vp, sz, vp]),
+        "w4a8_signal_ready": (st, [vp, vp]),
         "w4a8_nvfp4_scale_bytes": (sz, [i64, i64]),
         "w4a8_nvfp4_quantize": (st, [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, ctypes.c_int32,
                                      vp, vp, vp, vp, vp]),
@@ -445,6 +446,14 @@ def linear_flagged(x: torch.Tensor, packed: torch.Tensor, n: int, x_ready: torch
         x.data_ptr(), m, k, packed.data_ptr(), n, out.data_ptr(), x_ready.data_ptr(), workspace.data_ptr(),
         workspace.numel(), _stream(stream)))
     return out
+
+
+def signal_ready(x_ready: torch.Tensor, stream=None) -> None:
+    """Writes 1 to ``x_ready[0]`` in stream order (after the stream's earlier
+    work, e.g. the copy of x) without a host copy: w4a8_signal_ready."""
+    lib = load_library()
+    _cuda(x_ready, torch.int32, "x_ready")
+    _check("w4a8_signal_ready", lib.w4a8_signal_ready(x_ready.data_ptr(), _stream(stream)))
 
 
 # ---------------------------------------------------------------- NVFP4 comparison layer

@@ -6,6 +6,8 @@
 #include <new>
 #include <vector>
 
+#include <cuda.h>  // driver types for the stream write below (resolved at run time, not linked)
+
 #include "w4a8.h"
 
 #include "act.cuh"
@@ -551,6 +553,32 @@ w4a8_status w4a8_linear_flagged(const uint16_t* x, int64_t M, int64_t K, const v
   w4a8_status st = w4a8_linear_prepare(x, M, K, N, workspace, workspace_bytes, stream);
   if (st != W4A8_OK) return st;
   return w4a8_linear_run(M, K, packed, N, y, workspace, workspace_bytes, stream);
+}
+
+// cuStreamWriteValue32 of the driver, looked up once through the runtime
+// (the library links no driver library).  Null if the driver lacks it.
+using WriteValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+static WriteValue32Fn stream_write_value32() {
+  static const WriteValue32Fn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuStreamWriteValue32", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return WriteValue32Fn(nullptr);
+    return reinterpret_cast<WriteValue32Fn>(f);
+  }();
+  return fn;
+}
+
+w4a8_status w4a8_signal_ready(unsigned* x_ready, void* stream) {
+  if (!x_ready) return W4A8_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(x_ready) & 7u) return W4A8_ERR_ALIGN;
+  const WriteValue32Fn fn = stream_write_value32();
+  if (!fn) return W4A8_ERR_CUDA;
+  // default flags: the write is ordered after every earlier write of the stream
+  if (fn(static_cast<CUstream>(stream), reinterpret_cast<CUdeviceptr>(x_ready), 1u, 0u) != CUDA_SUCCESS)
+    return W4A8_ERR_CUDA;
+  return W4A8_OK;
 }
 
 // Device address of g_static_scratch, looked up once per device with that
