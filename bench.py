@@ -73,15 +73,36 @@ def strip_comments(src: str) -> str:
 
 def kernel_source_hash(files) -> str:
     """Hash of the comment-stripped kernel sources a traffic figure was
-    captured from."""
+    captured from.  An entry (file, marker) covers the file's stripped text
+    before `marker` only: the part a kernel compiles against when the rest
+    of the file holds other kernels (a missing marker is an error)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "w4a8_codebook_quantized_rotate_b200", "csrc", f)) as fh:
-            h.update(strip_comments(fh.read()).encode())
+        name, marker = f if isinstance(f, tuple) else (f, None)
+        with open(os.path.join(ROOT, "w4a8_codebook_quantized_rotate_b200", "csrc", name)) as fh:
+            text = strip_comments(fh.read())
+        if marker is not None:
+            cut = text.find(marker)
+            if cut < 0:
+                raise ValueError(f"{name}: marker not found")
+            text = text[:cut]
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, files) -> float | None:
+# The sources of each kernel with a committed traffic figure.  The one-token
+# kernel includes gemv.cuh for the helpers it shares with the multi-token
+# kernel, whose body (from decode_body on) it does not use.
+DECODE_MULTI_BODY = "template <int NB, int D, class Wait>\n__device__ __forceinline__ void decode_body"
+TRAFFIC_SOURCES = {
+    "decode_one_kernel_fused": ["gemv1.cuh", ("gemv.cuh", DECODE_MULTI_BODY), "act.cuh", "common.cuh"],
+    "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"],
+    "nvfp4_gemm_kernel_prefill": ["nvfp4.cuh", "act.cuh", "common.cuh"],
+    "gemm_sk_kernel_m128": ["gemm_sk.cuh", "gemm_tc.cuh", "common.cuh"],
+}
+
+
+def profiled_traffic(kernel: str, files=None) -> float | None:
     """DRAM bytes per launch from a committed ncu capture, if the kernel
     source is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -89,7 +110,7 @@ def profiled_traffic(kernel: str, files) -> float | None:
         return None
     with open(path) as f:
         d = json.load(f).get(kernel)
-    if not d or d.get("source_sha256_16") != kernel_source_hash(files):
+    if not d or d.get("source_sha256_16") != kernel_source_hash(files or TRAFFIC_SOURCES[kernel]):
         return None
     return float(d["dram_bytes_per_launch"])
 
@@ -432,8 +453,7 @@ def measure_c2(B, synth, torch, dev, rank, stream, steps, warmup):
                          "us_per_token": us / m, "TOPS": 2.0 * m * n * k / us / 1e6,
                          "path": c2_path(m, k, n)}
         if m == 128:  # the small-batch kernel's DRAM bytes from its committed capture at this size
-            out[f"M={m}"]["traffic"] = profiled_traffic("gemm_sk_kernel_m128",
-                                                        ["gemm_sk.cuh", "gemm_tc.cuh", "common.cuh"])
+            out[f"M={m}"]["traffic"] = profiled_traffic("gemm_sk_kernel_m128")
         del replay
     del copies
     torch.cuda.empty_cache()
@@ -779,8 +799,7 @@ def measure_nvfp4(B, torch, dev, rank, stream, peaks, steps=30, dec_steps=2000, 
                              "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
                              "peak_note": "measured dense bf16 burst peak x 4 (the nominal dense fp4/bf16 "
                                           "ratio, 9 / 2.25 PFLOP/s)",
-                             "traffic": profiled_traffic("nvfp4_gemm_kernel_prefill",
-                                                         ["nvfp4.cuh", "act.cuh", "common.cuh"]),
+                             "traffic": profiled_traffic("nvfp4_gemm_kernel_prefill"),
                              "ms_per_launch": gemm_ms}}
         else:
             gb = wbytes / (gemm_ms * 1e-3) / 1e9
@@ -1077,7 +1096,7 @@ def main() -> None:
             "kernel": "decode_one_kernel<true> (M=1, rotate + quantise fused)",
             "bound": "hbm", "achieved": step_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": step_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
-            "traffic": profiled_traffic("decode_one_kernel_fused", ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"]),
+            "traffic": profiled_traffic("decode_one_kernel_fused"),
             "us_per_launch": ms_step * 1e3,
             "note": "the step is this one kernel, so its launch duration is the step time",
         },
@@ -1093,7 +1112,7 @@ def main() -> None:
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": gemm_tflops / peaks["bf16_tflops"],
                          "peak_note": "measured dense bf16 burst peak; fp16 kind::f16 runs at the bf16 rate",
-                         "traffic": profiled_traffic("gemm_tc_kernel", ["gemm_tc.cuh", "common.cuh"]),
+                         "traffic": profiled_traffic("gemm_tc_kernel"),
                          "ms_per_launch": gemm_ms},
             "clocks": pre_clocks,
         },

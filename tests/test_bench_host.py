@@ -21,11 +21,7 @@ def test_weight_bytes_is_the_packed_layer():
 def test_committed_traffic_matches_its_source_hash():
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         d = json.load(f)
-    files = {"decode_one_kernel_fused": ["gemv1.cuh", "gemv.cuh", "act.cuh", "common.cuh"],
-             "gemm_tc_kernel": ["gemm_tc.cuh", "common.cuh"],
-             "nvfp4_gemm_kernel_prefill": ["nvfp4.cuh", "act.cuh", "common.cuh"],
-             "gemm_sk_kernel_m128": ["gemm_sk.cuh", "gemm_tc.cuh", "common.cuh"]}
-    for kernel, srcs in files.items():
+    for kernel, srcs in bench.TRAFFIC_SOURCES.items():
         if kernel not in d:
             assert bench.profiled_traffic(kernel, srcs) is None
             continue
@@ -37,6 +33,22 @@ def test_committed_traffic_matches_its_source_hash():
             assert got >= 17408 * 5120 * (0.5 + 1 / 16)
         else:
             assert got is None
+
+
+def test_one_token_hash_covers_the_shared_helpers_only():
+    """The one-token kernel's hash takes gemv.cuh up to the multi-token body:
+    the marker is there once, the part before it holds what the one-token
+    kernel uses (its parameters, its wait), and the body is outside it."""
+    with open(os.path.join(bench.ROOT, "w4a8_codebook_quantized_rotate_b200", "csrc", "gemv.cuh")) as f:
+        text = bench.strip_comments(f.read())
+    assert text.count(bench.DECODE_MULTI_BODY) == 1
+    head = text[:text.find(bench.DECODE_MULTI_BODY)]
+    assert "struct DecodeParams" in head and "struct DecWaitPdl" in head
+    assert "decode_body" not in head and "decode_kernel" not in head
+    gemv1 = open(os.path.join(bench.ROOT, "w4a8_codebook_quantized_rotate_b200", "csrc", "gemv1.cuh")).read()
+    assert "decode_body" not in bench.strip_comments(gemv1)  # the one-token kernel never calls it
+    with pytest.raises(ValueError):
+        bench.kernel_source_hash([("gemv.cuh", "no such text")])
 
 
 def test_traffic_is_withheld_when_the_source_changes(tmp_path, monkeypatch):

@@ -31,8 +31,10 @@
 // levels, both in a fixed order (the result is deterministic): the warps of
 // a CTA leave their partials in shared memory and one warp adds them after a
 // CTA barrier; a pair that also crosses into other CTAs leaves each CTA's
-// partial in the workspace, and the last CTA to finish (an atomic counter,
-// no waiting) adds them in CTA order and writes y.
+// partial in the workspace: between two CTAs each lane meets its counterpart
+// through an exchange word and the second to arrive adds the two; among
+// more, the last CTA to finish (an atomic counter, no waiting) adds them in
+// CTA order and writes y.
 #pragma once
 
 #include <type_traits>
@@ -609,6 +611,38 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const Wait& w
           const int tok = 8 * j + 2 * t + (e & 1);
           if (tok < p.M) mine[(i * 16 + g + 8 * (e >> 1)) * p.M + tok] = acc[i][j][e];
         }
+    if (cl == cf + 1) {
+      // Two CTAs: each lane meets its counterpart through one exchange word
+      // (the one-token kernel's words at this boundary).  The release orders
+      // the lane's partial before the word; the second lane to arrive adds
+      // the other's partial (a + b: the same in either order, and the same
+      // as the arrival-count path) and writes the lane's values.
+      unsigned long long* word = p.xch + size_t(cf) * 32 + lane;
+      unsigned long long other;
+      asm volatile("atom.acq_rel.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(other) : "l"(word), "l"(1ull) : "memory");
+      if (other == 0ull) continue;  // the other CTA finishes this lane's values
+      *word = 0ull;                 // ready for the next launch on this workspace
+      const int oc = int(blockIdx.x) == cf ? cl : cf;
+      const float* theirs = p.slots + size_t(oc * 2 + (dec_cta_begin<kW>(oc, p) >= q0 ? 0 : 1)) * sf;
+      float v[kDecTG][NB][4];
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i)
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = 8 * j + 2 * t + (e & 1);
+            v[i][j][e] = tok < p.M ? __ldcg(theirs + (i * 16 + g + 8 * (e >> 1)) * p.M + tok) : 0.f;
+          }
+#pragma unroll
+      for (int i = 0; i < kDecTG; ++i)
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[i][j][e] += v[i][j][e];
+      dec_epilogue<NB>(acc, p, pr, lane, ep);
+      continue;
+    }
     __threadfence();
     __syncwarp();
     unsigned old = 0;
