@@ -174,3 +174,35 @@ def test_static_scratch_holds_every_decode_plan(lib):
                for m in (1, 2, 8, 9, 16) for k in (256, 8192, 8448, 32768) for n in (16, 5120, 17408, 1 << 20))
     assert 0 < need <= size
     assert size <= 2 * need
+
+
+def test_header_is_plain_c_and_links_against_the_library(lib):
+    """include/w4a8.h is a C header: a C99 program (pedantic) that includes
+    it compiles, links against the built library by the declared names, and
+    runs a host-only entry (no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "_build", "abi_c")
+    os.makedirs(out_dir, exist_ok=True)
+    src = os.path.join(out_dir, "abi.c")
+    exe = os.path.join(out_dir, "abi")
+    with open(src, "w") as f:
+        f.write('#include <stdio.h>\n#include "w4a8.h"\n'
+                "int main(void) {\n"
+                "  size_t b = w4a8_packed_bytes(17408, 5120);\n"
+                "  size_t z = w4a8_packed_bytes(17408, 100);\n"
+                '  printf("%zu %zu %s\\n", b, z, w4a8_status_string(W4A8_ERR_SHAPE));\n'
+                "  return 0;\n"
+                "}\n")
+    from w4a8_codebook_quantized_rotate_b200 import binding
+    libdir = os.path.dirname(binding.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.dirname(HEADER),
+                    src, "-o", exe, "-L", libdir, "-lw4a8", "-Wl,-rpath," + libdir], check=True)
+    res = subprocess.run([exe], check=True, capture_output=True, text=True)
+    b, z, msg = res.stdout.split(" ", 2)
+    assert int(b) == 256 + 4 * 17408 + 17408 * 5120 // 2 + 17408 * 5120 // 16
+    assert int(z) == 0  # K not a multiple of 256: zero size
+    assert msg.strip() == lib.w4a8_status_string(2).decode()
